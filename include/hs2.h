@@ -1,0 +1,152 @@
+/*
+ * hs2.h -- C ABI of the HySparse2 hybrid sparse attention step on NVIDIA B200 (sm_100a).
+ *
+ * What the step computes
+ * ----------------------
+ * HySparse2 places hybrid sparse attention in the cross-decoder: a full-attention
+ * layer over the shared KV cache, followed by sparse layers ("HySparse2 Cuts the
+ * Prefill Path for Tool-Using Agents", section "One Cache Plan, Two Sharing Layers").
+ * Each sparse layer reuses that layer's KV cache and its per-token selection,
+ * and the most recent tokens are always part of the selection (KV Reuse; "HySparse2
+ * od Xiaomi zkracuje zpracovani dlouheho kontextu", section "Proc neni nutne znovu
+ * zpracovat cely dlouhy vstup", third paragraph; DAIR.AI newsletter, HySparse2
+ * bullets "Two levels of KV sharing" and "Prefill exits early").
+ *
+ * Notation: batch B, query heads Hq, kv heads Hkv, G = Hq / Hkv query heads per kv
+ * head (query head hq reads kv head hq / G), head dim d, cached tokens N, queries T
+ * per batch row, query position pos[b][t] (0 <= pos < N; key j is visible iff j <= pos),
+ * selection size k, forced window W, scale = d^-1/2.
+ *
+ *   full attention:   l_j = scale <q_full, k_j>,  LSE_full = ln sum_{j<=pos} e^{l_j},
+ *                     O_full = sum_{j<=pos} e^{l_j - LSE_full} v_j
+ *   selection score:  s_j = max over the G heads of kv head h of (l_j - LSE_full),
+ *                     for j in the pool [0, pos - W]   (the pages leave the score
+ *                     open; this library fixes it to the GQA-max log-softmax)
+ *   selection:        the min(k, |pool|) pool keys of largest s (ties: lower index)
+ *                     plus the window [max(0, pos - W + 1), pos]
+ *   sparse attention: the full-attention formula with Q_sparse over the selected
+ *                     keys only; all G heads of kv head h share the selection.
+ *
+ * Conventions (all entry points)
+ * ------------------------------
+ *  - Every tensor pointer is DEVICE memory owned by the caller, contiguous row-major
+ *    in the layout given, 16-byte aligned.  bf16 tensors are passed as const void*
+ *    holding IEEE bfloat16 bit patterns.
+ *      Q_full, Q_sparse, O_full, O_sparse : bf16  [B][Hq][T][d]
+ *      K, V                               : bf16  [B][Hkv][N][d]
+ *      pos                                : int32 [B][T]
+ *      LSE_full, LSE_sparse               : fp32  [B][Hq][T]   (natural log)
+ *      idx                                : int32 [B][Hkv][T][k + W]
+ *      cnt                                : int32 [B][Hkv][T]
+ *  - idx row r holds cnt[r] valid key indices followed by -1 padding.  The order of
+ *    the valid entries is unspecified (attention does not depend on key order).
+ *  - ws is a device workspace of at least hs2_workspace_size(dims) bytes, 256-byte
+ *    aligned, owned by the caller; its contents need no initialisation and are
+ *    overwritten by every call.  The library allocates no memory of its own.
+ *  - stream is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous on that stream: no host synchronisation, no device->host copy.
+ *  - Host-side argument checks run before any launch: a failing check returns an
+ *    error and launches nothing.  Launch failures return HS2_ERR_CUDA.
+ *  - Problems the host cannot see (a pos outside [0, N), an index outside [0, pos]
+ *    passed to hs2_sparse_attn, a non-finite score) set bits in a device status
+ *    word inside ws; kernels clamp or skip the offending element and continue.  Read
+ *    the word with hs2_read_device_status.  Each entry point clears it when it starts.
+ *  - Supported shapes: d in {64, 128}; G in {1, 2, 4, 8, 16}; B, Hq, Hkv, T, N >= 1;
+ *    T <= N; k >= 0; W >= 0; k + W < 2^31.  Anything else is HS2_ERR_UNSUPPORTED or
+ *    HS2_ERR_INVALID_ARG.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HS2_API __attribute__((visibility("default")))
+#else
+#define HS2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hs2_status {
+    HS2_OK = 0,
+    HS2_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned pointer, pos/shape mismatch */
+    HS2_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes (d, G) */
+    HS2_ERR_WORKSPACE = 3,    /* ws is null or smaller than hs2_workspace_size(dims), or misaligned */
+    HS2_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    HS2_ERR_DEVICE = 5        /* returned only by hs2_read_device_status when status bits are set */
+} hs2_status;
+
+/* Bits of the device status word (see hs2_read_device_status). */
+#define HS2_DEV_BAD_POS       0x1u  /* a pos[b][t] outside [0, N): clamped into range */
+#define HS2_DEV_BAD_INDEX     0x2u  /* hs2_sparse_attn got an index outside [0, pos]: key skipped */
+#define HS2_DEV_NONFINITE     0x4u  /* a selection score was NaN: ranked below every finite score */
+#define HS2_DEV_TIMEOUT       0x8u  /* a pipeline wait exceeded its bound: kernel gave up, outputs invalid */
+#define HS2_DEV_CAND_OVERFLOW 0x10u /* informational: top-k threshold bucket overflowed its buffer; slow exact path used */
+
+/* Problem shape.  The attention scale is fixed to d^-1/2. */
+typedef struct hs2_dims {
+    int32_t B, Hq, Hkv, T, N, d, k, W;
+} hs2_dims;
+
+/* Bytes of device workspace every entry point below needs for these dims (a multiple of
+ * 256).  Returns 0 if the dims are invalid or unsupported.  Pure host computation. */
+HS2_API size_t hs2_workspace_size(const hs2_dims* dims);
+
+/* Full-attention layer: O_full and LSE_full for every (b, hq, t), keys 0..pos[b][t].
+ * Source: the full-attention layer of the hybrid block ("HySparse2 Cuts the Prefill
+ * Path...", "One Cache Plan, Two Sharing Layers"); split-K flash-decode with a
+ * log-sum-exp combine (as in "Simplified Sparse Attention via Gist Tokens", section
+ * 3.6, "three-kernel split-K sparse flash-decode"). */
+HS2_API hs2_status hs2_full_attn(const hs2_dims* dims, const void* Q_full, const void* K, const void* V,
+                         const int32_t* pos, void* O_full, float* LSE_full,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Token-level selection: scores every pool key with the GQA-max log-softmax score (using
+ * the caller's LSE_full, as produced by hs2_full_attn), keeps the min(k, |pool|) best
+ * (ties to the lower index) and adds the forced window.  Writes idx and cnt
+ * (cnt = min(k, |pool|) + min(W, pos + 1)).  Source: token-level selection with forced
+ * recent tokens ("HySparse2 od Xiaomi...", third paragraph; DAIR.AI newsletter,
+ * "Prefill exits early"). */
+HS2_API hs2_status hs2_select(const hs2_dims* dims, const void* Q_full, const void* K,
+                      const float* LSE_full, const int32_t* pos, int32_t* idx, int32_t* cnt,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Sparse layer with KV Reuse: attention of Q_sparse over the keys listed in idx/cnt
+ * (the same list for all G query heads of a kv head).  Any idx/cnt the caller supplies
+ * is accepted; entries outside [0, pos] are skipped and flag HS2_DEV_BAD_INDEX, and
+ * cnt is clamped to [0, k + W].  A row with no keys gives O = 0, LSE = -inf.
+ * Source: KV Reuse ("HySparse2 od Xiaomi...", third paragraph; DAIR.AI newsletter,
+ * "Two levels of KV sharing"). */
+HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, const void* K,
+                           const void* V, const int32_t* pos, const int32_t* idx,
+                           const int32_t* cnt, void* O_sparse, float* LSE_sparse,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* The whole hybrid step: hs2_full_attn, hs2_select and hs2_sparse_attn in order on one
+ * stream, sharing intermediates through ws (when T*G <= 16 the full-attention pass
+ * also keeps its logits so the selection does not read K a second time). */
+HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
+                    const void* K, const void* V, const int32_t* pos,
+                    void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,
+                    int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream);
+
+/* Copies the device status word out of ws and waits for the stream (the only synchronising
+ * call).  *bits receives the HS2_DEV_* bits; returns HS2_ERR_DEVICE if any bit other than
+ * HS2_DEV_CAND_OVERFLOW is set, else HS2_OK. */
+HS2_API hs2_status hs2_read_device_status(const void* ws, void* stream, uint32_t* bits);
+
+/* Static, human-readable name of a status code. */
+HS2_API const char* hs2_status_string(hs2_status status);
+
+/* Library version, (major << 16) | minor. */
+HS2_API uint32_t hs2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H_ */

@@ -1,0 +1,210 @@
+// Warp-level attention on one 16-row query tile against a shared-memory K/V tile.
+//
+// The query rows of one kv head (its G query heads, for one or more queries) form
+// 16-row tiles.  A warp owns one such tile and a slice of KW keys of the current
+// 64-key K/V tile, computes S = Q K^T with bf16 mma.sync (fp32 accumulate), applies
+// the causal / validity mask, and folds the slice into a running online softmax
+// (m, l, O) in base-2 units: logits are pre-multiplied by d^-1/2 * log2(e) so every
+// exponential is one ex2.  The split-K partial results (m, l, O) merge exactly with
+// the log-sum-exp correction, as in the split-K flash-decode of "Simplified Sparse
+// Attention via Gist Tokens", section 3.6 ("three-kernel split-K sparse flash-decode").
+//
+// Register fragments follow the m16n8k16 layout: lane = 4*g + c holds rows g and g+8
+// and, per 8-key n-tile, columns 2c and 2c+1.
+#pragma once
+
+#include "hs2_device.cuh"
+
+namespace hs2 {
+
+// A fragments of a 16 x D bf16 query tile (row-major), kept in registers for the whole sweep.
+template <int D>
+struct QTile {
+    uint32_t a[D / 16][4];
+
+    // rows: global element offsets of tile rows g and g+8 for this lane (-1 = padding row)
+    __device__ __forceinline__ void load(const uint16_t* __restrict__ Q, int64_t off_lo, int64_t off_hi) {
+        const int c = threadIdx.x & 3;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int col = kk * 16 + 2 * c;
+            a[kk][0] = off_lo >= 0 ? *reinterpret_cast<const uint32_t*>(Q + off_lo + col) : 0u;
+            a[kk][1] = off_hi >= 0 ? *reinterpret_cast<const uint32_t*>(Q + off_hi + col) : 0u;
+            a[kk][2] = off_lo >= 0 ? *reinterpret_cast<const uint32_t*>(Q + off_lo + col + 8) : 0u;
+            a[kk][3] = off_hi >= 0 ? *reinterpret_cast<const uint32_t*>(Q + off_hi + col + 8) : 0u;
+        }
+    }
+};
+
+// S[16 x KW] = Q[16 x D] * K[key0 .. key0+KW)^T, K read from a swizzled tile at smem address kbase.
+template <int D, int KW>
+__device__ __forceinline__ void qk_tile(const QTile<D>& q, uint32_t kbase, int key0, float (&s)[KW / 8][4]) {
+    const int lane = threadIdx.x & 31;
+    const int mi = lane >> 3;
+#pragma unroll
+    for (int n = 0; n < KW / 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+    for (int kg = 0; kg < KW / 16; ++kg) {
+        const int row = key0 + kg * 16 + (lane & 7) + ((mi >> 1) << 3);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kbase + tile_chunk_offset(row, 2 * kk + (mi & 1)), b0, b1, b2, b3);
+            mma_bf16(s[2 * kg], q.a[kk], b0, b1);
+            mma_bf16(s[2 * kg + 1], q.a[kk], b2, b3);
+        }
+    }
+}
+
+// Running softmax state of one warp's 16-row tile.
+template <int D>
+struct OnlineSoftmax {
+    float o[D / 8][4];
+    float m[2];  // running max (base-2 logits) of rows g, g+8
+    float l[2];  // this lane's partial sum of 2^(logit - m) (summed over the quad at the end)
+
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        m[0] = m[1] = -INFINITY;
+        l[0] = l[1] = 0.f;
+    }
+
+    // Fold in a slice of base-2 logits s (already masked with -inf); V from the swizzled tile at vbase.
+    template <int KW>
+    __device__ __forceinline__ void update(float (&s)[KW / 8][4], uint32_t vbase, int key0) {
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int n = 0; n < KW / 8; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * ri], s[n][2 * ri + 1]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m[ri], mx);
+            const float base = (m_new == -INFINITY) ? 0.f : m_new;
+            const float corr = fast_exp2(m[ri] - base);
+            float sum = 0.f;
+#pragma unroll
+            for (int n = 0; n < KW / 8; ++n) {
+                s[n][2 * ri] = fast_exp2(s[n][2 * ri] - base);
+                s[n][2 * ri + 1] = fast_exp2(s[n][2 * ri + 1] - base);
+                sum += s[n][2 * ri] + s[n][2 * ri + 1];
+            }
+            l[ri] = l[ri] * corr + sum;
+            m[ri] = m_new;
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) {
+                o[n][2 * ri] *= corr;
+                o[n][2 * ri + 1] *= corr;
+            }
+        }
+        // O += P V
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int kg = 0; kg < KW / 16; ++kg) {
+            uint32_t a[4];
+            a[0] = pack_bf16x2(s[2 * kg][0], s[2 * kg][1]);
+            a[1] = pack_bf16x2(s[2 * kg][2], s[2 * kg][3]);
+            a[2] = pack_bf16x2(s[2 * kg + 1][0], s[2 * kg + 1][1]);
+            a[3] = pack_bf16x2(s[2 * kg + 1][2], s[2 * kg + 1][3]);
+            const int row = key0 + kg * 16 + (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+            for (int dn = 0; dn < D / 16; ++dn) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vbase + tile_chunk_offset(row, 2 * dn + (mi >> 1)), b0, b1, b2, b3);
+                mma_bf16(o[2 * dn], a, b0, b1);
+                mma_bf16(o[2 * dn + 1], a, b2, b3);
+            }
+        }
+    }
+
+    // Sum l over the 4 lanes of each row.
+    __device__ __forceinline__ void finish_rows() {
+#pragma unroll
+        for (int ri = 0; ri < 2; ++ri) {
+            l[ri] += __shfl_xor_sync(0xffffffffu, l[ri], 1);
+            l[ri] += __shfl_xor_sync(0xffffffffu, l[ri], 2);
+        }
+    }
+};
+
+// Split-K partial of one row: (m, l) in base-2 units and the unnormalised O.
+struct PartialRef {
+    float2* ml;   // [rows] (m, l)
+    float* acc;   // [rows][D]
+};
+
+// Write a warp's tile straight to the partial buffers (one warp per tile, no merge).
+// row_out(r) gives the global partial row of tile row r, or -1 to skip it.
+template <int D, class RowOut>
+__device__ __forceinline__ void store_partial(const OnlineSoftmax<D>& st, const PartialRef& out, RowOut row_out) {
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int ri = 0; ri < 2; ++ri) {
+        const int grow = row_out(g + 8 * ri);
+        if (grow < 0) continue;
+        float* dst = out.acc + static_cast<int64_t>(grow) * D;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n)
+            *reinterpret_cast<float2*>(dst + n * 8 + 2 * c) = make_float2(st.o[n][2 * ri], st.o[n][2 * ri + 1]);
+        if (c == 0) out.ml[grow] = make_float2(st.m[ri], st.l[ri]);
+    }
+}
+
+// Shared scratch for merging the NKS warps that swept disjoint key slices of one tile.
+template <int D>
+constexpr int merge_ld() { return D + 4; }
+template <int D, int NKS>
+constexpr int merge_floats() { return NKS * 16 * (merge_ld<D>() + 2); }
+
+// Phase 1 (every warp of the tile): park this warp's state in shared memory slot ks.
+template <int D, int NKS>
+__device__ __forceinline__ void stash_state(const OnlineSoftmax<D>& st, int ks, float* red) {
+    constexpr int LD = merge_ld<D>();
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    float* red_ml = red + NKS * 16 * LD;
+#pragma unroll
+    for (int ri = 0; ri < 2; ++ri) {
+        const int r = g + 8 * ri;
+        float* dst = red + (ks * 16 + r) * LD;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n)
+            *reinterpret_cast<float2*>(dst + n * 8 + 2 * c) = make_float2(st.o[n][2 * ri], st.o[n][2 * ri + 1]);
+        if (c == 0) {
+            red_ml[(ks * 16 + r) * 2] = st.m[ri];
+            red_ml[(ks * 16 + r) * 2 + 1] = st.l[ri];
+        }
+    }
+}
+
+// Phase 2 (after a barrier; threads tid = 0..nthr-1 of the tile): merge the NKS states
+// with the log-sum-exp correction and write the tile's partial.
+template <int D, int NKS, class RowOut>
+__device__ __forceinline__ void merge_states(const float* red, int tid, int nthr, const PartialRef& out,
+                                             RowOut row_out) {
+    constexpr int LD = merge_ld<D>();
+    const float* red_ml = red + NKS * 16 * LD;
+    for (int e = tid; e < 16 * D; e += nthr) {
+        const int r = e / D, dcol = e % D;
+        const int grow = row_out(r);
+        if (grow < 0) continue;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NKS; ++w) M = fmaxf(M, red_ml[(w * 16 + r) * 2]);
+        float L = 0.f, A = 0.f;
+#pragma unroll
+        for (int w = 0; w < NKS; ++w) {
+            const float mw = red_ml[(w * 16 + r) * 2];
+            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+            L += f * red_ml[(w * 16 + r) * 2 + 1];
+            A += f * red[(w * 16 + r) * LD + dcol];
+        }
+        out.acc[static_cast<int64_t>(grow) * D + dcol] = A;
+        if (dcol == 0) out.ml[grow] = make_float2(M, L);
+    }
+}
+
+}  // namespace hs2

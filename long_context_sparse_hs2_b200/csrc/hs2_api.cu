@@ -1,0 +1,329 @@
+// C ABI of the HySparse2 hybrid sparse attention step: argument checks, the execution
+// plan (grids, split factors, workspace layout), TMA descriptors and launch order.
+// Declared and documented in include/hs2.h.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "hs2_internal.h"
+
+namespace hs2 {
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Split-K factor minimising (waves x tiles per split), with a tiny penalty per split.
+int choose_splits(int64_t units, int64_t tiles, int64_t slots, int max_splits) {
+    int best = 1;
+    double best_cost = 1e300;
+    const int limit = static_cast<int>(std::min<int64_t>(max_splits, std::max<int64_t>(tiles, 1)));
+    for (int s = 1; s <= limit; ++s) {
+        const int64_t waves = (units * s + slots - 1) / slots;
+        const int64_t per = (tiles + s - 1) / s;
+        const double cost = static_cast<double>(waves * per) + 0.01 * s;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+
+bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
+    *why = HS2_ERR_INVALID_ARG;
+    if (!dm) return false;
+    const hs2_dims& x = *dm;
+    if (x.B < 1 || x.Hq < 1 || x.Hkv < 1 || x.T < 1 || x.N < 1 || x.k < 0 || x.W < 0) return false;
+    if (x.T > x.N || x.Hq % x.Hkv != 0) return false;
+    if (static_cast<int64_t>(x.k) + x.W >= (int64_t(1) << 31)) return false;
+    const int64_t rows_q = static_cast<int64_t>(x.B) * x.Hq * x.T;
+    const int64_t rows_kv = static_cast<int64_t>(x.B) * x.Hkv * x.T;
+    if (rows_q >= (int64_t(1) << 31) || static_cast<int64_t>(x.B) * x.Hkv >= (int64_t(1) << 31)) return false;
+    *why = HS2_ERR_UNSUPPORTED;
+    const int G = x.Hq / x.Hkv;
+    if (x.d != 64 && x.d != 128) return false;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return false;
+    if (rows_kv > 65535) return false;  // grid.y of the per-row kernels
+
+    Plan& P = *p;
+    P.B = x.B; P.Hq = x.Hq; P.Hkv = x.Hkv; P.T = x.T; P.N = x.N; P.d = x.d; P.k = x.k; P.W = x.W; P.G = G;
+    P.rows_q = rows_q;
+    P.rows_kv = rows_kv;
+    const int64_t rows = static_cast<int64_t>(x.T) * G;
+    P.RT = 1;
+    while (P.RT < 8 && 16 * P.RT < rows) P.RT *= 2;
+    P.TQ = 16 * P.RT / G;
+    P.QB = (x.T + P.TQ - 1) / P.TQ;
+    P.mat_logits = (P.RT == 1 && P.QB == 1);
+    const int64_t units = static_cast<int64_t>(x.B) * x.Hkv * P.QB;
+    if (units > 65535) return false;  // grid.y of the streaming kernels
+    const int64_t tiles = (x.N + kKeyTile - 1) / kKeyTile;
+    const int64_t slots = (P.RT == 1 ? 2 : 1) * int64_t(kSMs);
+    P.S1 = choose_splits(units, tiles, slots, 256);
+
+    const int64_t kw = static_cast<int64_t>(x.k) + x.W;
+    P.C4 = 1024;
+    while (P.C4 > 64 && rows_kv * ((kw + P.C4 - 1) / P.C4) < 4 * kSMs) P.C4 /= 2;
+    P.S4 = static_cast<int>(std::max<int64_t>(1, (kw + P.C4 - 1) / P.C4));
+    P.cand_cap = std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
+
+    size_t off = 0;
+    P.off_status = off; off += 256;
+    P.off_meta = off; off = align_up(off + rows_kv * kMetaInts * 4, 256);
+    P.off_hist = off; off = align_up(off + rows_kv * kHistBins * 4, 256);
+    P.zero_bytes = off;
+    P.off_pf_ml = off; off = align_up(off + size_t(P.S1) * rows_q * 8, 256);
+    P.off_pf_acc = off; off = align_up(off + size_t(P.S1) * rows_q * x.d * 4, 256);
+    P.off_ps_ml = off; off = align_up(off + size_t(P.S4) * rows_q * 8, 256);
+    P.off_ps_acc = off; off = align_up(off + size_t(P.S4) * rows_q * x.d * 4, 256);
+    P.off_keys = off; off = align_up(off + size_t(rows_kv) * x.N * 4, 256);
+    P.off_cand = off; off = align_up(off + size_t(rows_kv) * P.cand_cap * 8, 256);
+    P.off_logits = off;
+    if (P.mat_logits) off = align_up(off + size_t(rows_kv) * x.N * G * 4, 256);
+    P.total = off;
+    *why = HS2_OK;
+    return true;
+}
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 3-D view [B*Hkv][N][d] of a K or V cache; 64 x 64 boxes, 128-byte swizzle, zero fill out of range.
+bool make_kv_map(CUtensorMap* m, const void* base, const Plan& p) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(p.d), cuuint64_t(p.N), cuuint64_t(p.B) * p.Hkv};
+    const cuuint64_t strides[2] = {cuuint64_t(p.d) * 2, cuuint64_t(p.N) * p.d * 2};
+    const cuuint32_t box[3] = {64, cuuint32_t(kKeyTile), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Ws {
+    uint8_t* base;
+    template <class T>
+    T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+};
+
+hs2_status check_ws(const Plan& p, void* ws, size_t ws_bytes) {
+    if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return HS2_ERR_WORKSPACE;
+    return HS2_OK;
+}
+
+hs2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA; }
+
+#define HS2_TRY(expr)                                 \
+    do {                                              \
+        const hs2_status s_ = cuda_status(expr);      \
+        if (s_ != HS2_OK) return s_;                  \
+    } while (0)
+
+float scale_log2(const Plan& p) { return kLog2e / sqrtf(static_cast<float>(p.d)); }
+
+AttnArgs attn_args(const Plan& p, const void* Q, const int32_t* pos, const Ws& w) {
+    AttnArgs a{};
+    a.Q = static_cast<const uint16_t*>(Q);
+    a.pos = pos;
+    a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.T = p.T; a.N = p.N; a.G = p.G; a.W = p.W;
+    a.TQ = p.TQ; a.QB = p.QB; a.S = p.S1;
+    a.scale_log2 = scale_log2(p);
+    a.part_ml = w.at<float2>(p.off_pf_ml);
+    a.part_acc = w.at<float>(p.off_pf_acc);
+    a.status = w.at<unsigned>(p.off_status);
+    return a;
+}
+
+hs2_status run_full(const Plan& p, const void* Qf, const void* K, const void* V, const int32_t* pos, void* O_full,
+                    float* LSE_full, const Ws& w, bool keep_logits, cudaStream_t st) {
+    CUtensorMap tmK, tmV;
+    if (!make_kv_map(&tmK, K, p) || !make_kv_map(&tmV, V, p)) return HS2_ERR_CUDA;
+    AttnArgs a = attn_args(p, Qf, pos, w);
+    a.logits = keep_logits ? w.at<float>(p.off_logits) : nullptr;
+    HS2_TRY(launch_full_attn(p, tmK, tmV, a, st));
+    CombineArgs c{a.part_ml, a.part_acc, p.S1, p.rows_q, static_cast<uint16_t*>(O_full), LSE_full};
+    HS2_TRY(launch_combine(p.d, c, st));
+    return HS2_OK;
+}
+
+hs2_status run_select(const Plan& p, const void* Qf, const void* K, const float* LSE_full, const int32_t* pos,
+                      int32_t* idx, int32_t* cnt, const Ws& w, bool from_logits, cudaStream_t st) {
+    unsigned* status = w.at<unsigned>(p.off_status);
+    uint32_t* keys = w.at<uint32_t>(p.off_keys);
+    if (from_logits) {
+        ScoreArgs s{w.at<float>(p.off_logits), LSE_full, pos, p.B, p.Hq, p.Hkv, p.T, p.N, p.G, p.W, keys, status};
+        HS2_TRY(launch_score_from_logits(p, s, st));
+    } else {
+        CUtensorMap tmK;
+        if (!make_kv_map(&tmK, K, p)) return HS2_ERR_CUDA;
+        AttnArgs a = attn_args(p, Qf, pos, w);
+        a.lse = LSE_full;
+        a.keys = keys;
+        HS2_TRY(launch_score_sweep(p, tmK, a, st));
+    }
+    TopkArgs t{};
+    t.keys = keys;
+    t.pos = pos;
+    t.Hkv = p.Hkv; t.T = p.T; t.N = p.N; t.k = p.k; t.W = p.W;
+    t.rows = p.rows_kv;
+    t.hist = w.at<unsigned>(p.off_hist);
+    t.meta = w.at<int>(p.off_meta);
+    t.cand = w.at<unsigned long long>(p.off_cand);
+    t.cand_cap = p.cand_cap;
+    t.idx = idx;
+    t.cnt = cnt;
+    t.status = status;
+    HS2_TRY(launch_topk(p, t, st));
+    return HS2_OK;
+}
+
+hs2_status run_sparse(const Plan& p, const void* Qs, const void* K, const void* V, const int32_t* pos,
+                      const int32_t* idx, const int32_t* cnt, void* O_sparse, float* LSE_sparse, const Ws& w,
+                      cudaStream_t st) {
+    SparseArgs s{};
+    s.Q = static_cast<const uint16_t*>(Qs);
+    s.K = static_cast<const uint16_t*>(K);
+    s.V = static_cast<const uint16_t*>(V);
+    s.pos = pos;
+    s.idx = idx;
+    s.cnt = cnt;
+    s.B = p.B; s.Hq = p.Hq; s.Hkv = p.Hkv; s.T = p.T; s.N = p.N; s.G = p.G; s.kw = p.k + p.W;
+    s.C4 = p.C4; s.S4 = p.S4;
+    s.scale_log2 = scale_log2(p);
+    s.part_ml = w.at<float2>(p.off_ps_ml);
+    s.part_acc = w.at<float>(p.off_ps_acc);
+    s.status = w.at<unsigned>(p.off_status);
+    HS2_TRY(launch_sparse_attn(p, s, st));
+    CombineArgs c{s.part_ml, s.part_acc, p.S4, p.rows_q, static_cast<uint16_t*>(O_sparse), LSE_sparse};
+    HS2_TRY(launch_combine(p.d, c, st));
+    return HS2_OK;
+}
+
+bool ok16(const void* p) { return p && aligned(p, 16); }
+bool ok4(const void* p) { return p && aligned(p, 4); }
+
+}  // namespace
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+size_t hs2_workspace_size(const hs2_dims* dims) {
+    Plan p;
+    hs2_status why;
+    return make_plan(dims, &p, &why) ? p.total : 0;
+}
+
+hs2_status hs2_full_attn(const hs2_dims* dims, const void* Q_full, const void* K, const void* V, const int32_t* pos,
+                         void* O_full, float* LSE_full, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    hs2_status why;
+    if (!make_plan(dims, &p, &why)) return why;
+    if (!ok16(Q_full) || !ok16(K) || !ok16(V) || !ok4(pos) || !ok16(O_full) || !ok4(LSE_full))
+        return HS2_ERR_INVALID_ARG;
+    if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Ws w{static_cast<uint8_t*>(ws)};
+    HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));
+    return run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, false, st);
+}
+
+hs2_status hs2_select(const hs2_dims* dims, const void* Q_full, const void* K, const float* LSE_full,
+                      const int32_t* pos, int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    hs2_status why;
+    if (!make_plan(dims, &p, &why)) return why;
+    if (!ok16(Q_full) || !ok16(K) || !ok4(LSE_full) || !ok4(pos) || !ok4(idx) || !ok4(cnt))
+        return HS2_ERR_INVALID_ARG;
+    if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Ws w{static_cast<uint8_t*>(ws)};
+    HS2_TRY(cudaMemsetAsync(ws, 0, p.zero_bytes, st));
+    return run_select(p, Q_full, K, LSE_full, pos, idx, cnt, w, false, st);
+}
+
+hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, const void* K, const void* V,
+                           const int32_t* pos, const int32_t* idx, const int32_t* cnt, void* O_sparse,
+                           float* LSE_sparse, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    hs2_status why;
+    if (!make_plan(dims, &p, &why)) return why;
+    if (!ok16(Q_sparse) || !ok16(K) || !ok16(V) || !ok4(pos) || !ok4(idx) || !ok4(cnt) || !ok16(O_sparse) ||
+        !ok4(LSE_sparse))
+        return HS2_ERR_INVALID_ARG;
+    if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Ws w{static_cast<uint8_t*>(ws)};
+    HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));
+    return run_sparse(p, Q_sparse, K, V, pos, idx, cnt, O_sparse, LSE_sparse, w, st);
+}
+
+hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse, const void* K, const void* V,
+                    const int32_t* pos, void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,
+                    int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+    Plan p;
+    hs2_status why;
+    if (!make_plan(dims, &p, &why)) return why;
+    if (!ok16(Q_full) || !ok16(Q_sparse) || !ok16(K) || !ok16(V) || !ok4(pos) || !ok16(O_full) ||
+        !ok16(O_sparse) || !ok4(LSE_full) || !ok4(LSE_sparse) || !ok4(idx) || !ok4(cnt))
+        return HS2_ERR_INVALID_ARG;
+    if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Ws w{static_cast<uint8_t*>(ws)};
+    HS2_TRY(cudaMemsetAsync(ws, 0, p.zero_bytes, st));
+    hs2_status s = run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, p.mat_logits, st);
+    if (s != HS2_OK) return s;
+    s = run_select(p, Q_full, K, LSE_full, pos, idx, cnt, w, p.mat_logits, st);
+    if (s != HS2_OK) return s;
+    return run_sparse(p, Q_sparse, K, V, pos, idx, cnt, O_sparse, LSE_sparse, w, st);
+}
+
+hs2_status hs2_read_device_status(const void* ws, void* stream, uint32_t* bits) {
+    if (!ws || !bits || !aligned(ws, 256)) return HS2_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    HS2_TRY(cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st));
+    HS2_TRY(cudaStreamSynchronize(st));
+    *bits = v;
+    return (v & ~HS2_DEV_CAND_OVERFLOW) ? HS2_ERR_DEVICE : HS2_OK;
+}
+
+const char* hs2_status_string(hs2_status s) {
+    switch (s) {
+        case HS2_OK: return "ok";
+        case HS2_ERR_INVALID_ARG: return "invalid argument";
+        case HS2_ERR_UNSUPPORTED: return "unsupported shape";
+        case HS2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case HS2_ERR_CUDA: return "CUDA error";
+        case HS2_ERR_DEVICE: return "device status bits set";
+    }
+    return "unknown status";
+}
+
+uint32_t hs2_version(void) { return (1u << 16) | 0u; }
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+// Internal (host + device) declarations of the HySparse2 library: the execution plan of
+// one call, kernel argument blocks, and the host launchers each kernel file exports.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "hs2.h"
+
+namespace hs2 {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kKeyTile = 64;                      // keys per K/V shared-memory tile
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bound on any single pipeline wait (2 s)
+constexpr int kSMs = 148;            // B200 streaming multiprocessors
+constexpr int kHistBins = 8192;      // top-k histogram: 1/128 of a base-2 score unit per bin
+constexpr float kBinsPerUnit = 128.f;
+constexpr int kTopkChunk = 4096;     // pool keys per CTA in the histogram / emit passes
+constexpr int kMetaInts = 8;         // per-row top-k bookkeeping ints (see TopkMeta)
+
+// Per-row top-k bookkeeping in the workspace (ints; zeroed at the start of every call).
+enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDone = 2, kMetaDef = 3, kMetaCand = 4 };
+
+// Everything one call needs to know about shapes, grids and workspace offsets.
+struct Plan {
+    int B, Hq, Hkv, T, N, d, k, W, G;
+    int64_t rows_q;     // B*Hq*T   query-head rows
+    int64_t rows_kv;    // B*Hkv*T  selection rows
+    int RT;             // 16-row MMA tiles per attention row block (1, 2, 4, 8)
+    int TQ;             // queries per row block = 16*RT/G
+    int QB;             // row blocks per (b, kv head) = ceil(T / TQ)
+    int S1;             // split-K factor of the full-attention sweep
+    bool mat_logits;    // hs2_step keeps the full layer's logits instead of re-reading K
+    int C4;             // selected keys per sparse-attention CTA
+    int S4;             // sparse-attention splits per row = ceil((k+W)/C4)
+    int64_t cand_cap;   // per-row capacity of the top-k candidate buffer
+    // workspace byte offsets
+    size_t off_status, off_meta, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand,
+        off_logits, zero_bytes, total;
+};
+
+bool make_plan(const hs2_dims* dims, Plan* p, hs2_status* why);
+
+// ------------------------------------------------------------------ kernel arguments
+
+struct AttnArgs {
+    const uint16_t* Q;     // [B][Hq][T][D]
+    const int32_t* pos;    // [B][T]
+    int B, Hq, Hkv, T, N, G, W;
+    int TQ, QB, S;
+    float scale_log2;      // d^-1/2 * log2(e)
+    float2* part_ml;       // [S][rows_q]
+    float* part_acc;       // [S][rows_q][D]
+    float* logits;         // optional [rows_kv][N][G] base-2 logits (full sweep only)
+    const float* lse;      // [rows_q] natural-log LSE_full (score sweep only)
+    uint32_t* keys;        // [rows_kv][N] order-preserving score keys (score sweep only)
+    unsigned* status;
+};
+
+struct SparseArgs {
+    const uint16_t* Q;     // Q_sparse [B][Hq][T][D]
+    const uint16_t* K;     // [B][Hkv][N][D]
+    const uint16_t* V;
+    const int32_t* pos;    // [B][T]
+    const int32_t* idx;    // [rows_kv][k+W]
+    const int32_t* cnt;    // [rows_kv]
+    int B, Hq, Hkv, T, N, G, kw;  // kw = k + W (row stride of idx)
+    int C4, S4;
+    float scale_log2;
+    float2* part_ml;       // [S4][rows_q]
+    float* part_acc;       // [S4][rows_q][D]
+    unsigned* status;
+};
+
+struct CombineArgs {
+    const float2* part_ml;
+    const float* part_acc;
+    int S;
+    int64_t rows;
+    uint16_t* O;           // bf16 [rows][D]
+    float* LSE;            // [rows] natural log
+};
+
+struct ScoreArgs {         // scores from kept logits
+    const float* logits;   // [rows_kv][N][G]
+    const float* lse;      // [rows_q] natural log
+    const int32_t* pos;
+    int B, Hq, Hkv, T, N, G, W;
+    uint32_t* keys;        // [rows_kv][N]
+    unsigned* status;
+};
+
+struct TopkArgs {
+    const uint32_t* keys;  // [rows][N]
+    const int32_t* pos;    // [B][T]
+    int Hkv, T, N, k, W;
+    int64_t rows;
+    unsigned* hist;        // [rows][kHistBins]
+    int* meta;             // [rows][kMetaInts]
+    unsigned long long* cand;  // [rows][cand_cap] composite (key << 32 | ~index)
+    int64_t cand_cap;
+    int32_t* idx;          // [rows][k+W]
+    int32_t* cnt;          // [rows]
+    unsigned* status;
+};
+
+// ------------------------------------------------------------------ launchers (return cudaGetLastError())
+
+cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
+                             cudaStream_t st);
+cudaError_t launch_score_sweep(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_score_from_logits(const Plan& p, const ScoreArgs& a, cudaStream_t st);
+cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st);
+cudaError_t launch_topk(const Plan& p, const TopkArgs& a, cudaStream_t st);
+
+}  // namespace hs2

@@ -1,0 +1,164 @@
+// Sparse layer with KV Reuse: attention of Q_sparse over the selected keys only (sm_100a).
+//
+// Each sparse layer of a hybrid block reuses the preceding full-attention layer's KV
+// cache and its token selection ("HySparse2 od Xiaomi zkracuje zpracovani dlouheho
+// kontextu", section "Proc neni nutne znovu zpracovat cely dlouhy vstup", third
+// paragraph; DAIR.AI newsletter, HySparse2 bullet "Two levels of KV sharing").  All G
+// query heads of a kv head share one index list, so a CTA gathers each selected K/V row
+// once into shared memory and reuses it for the G heads -- the group-shared tile idea of
+// "Simplified Sparse Attention via Gist Tokens", section 3.3 ("Grouped Unfolding for GQA")
+// and section 3.6 (split-K partial attention over a compact list).
+//
+// Grid: (S4 splits, B*Hkv*T rows).  A CTA reads its C4 slots of the row's index list,
+// validates them (0 <= j <= pos; others are skipped and flagged), gathers the rows with
+// 16-byte cp.async into the same 128-byte-swizzled tile layout the TMA path uses,
+// double-buffered 64 keys at a time, and runs the shared warp attention core.  Splits
+// merge in combine_kernel.
+#include "attn_core.cuh"
+#include "hs2_internal.h"
+
+namespace hs2 {
+
+namespace {
+
+constexpr int kSparseWarps = 4;
+constexpr int kSparseThreads = kSparseWarps * 32;
+
+template <int D>
+struct SparseSmem {
+    static constexpr int kTileBytes = kKeyTile * D * 2;
+    static constexpr int kStageBytes = 2 * kTileBytes;  // K + V
+    static constexpr int kRingBytes = 2 * kStageBytes;
+    static constexpr int kIdxOff = kRingBytes;
+    static constexpr int bytes(int C4) { return kIdxOff + (C4 + kKeyTile) * 4 + 1024; }
+};
+
+template <int D>
+__device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_idx, int tile, uint8_t* stage,
+                                            int64_t kv_base) {
+    constexpr int CH = D / 8;                 // 16-byte chunks per row
+    constexpr int PER_T = kKeyTile * CH;      // chunks per tensor per tile
+    for (int ch = threadIdx.x; ch < 2 * PER_T; ch += kSparseThreads) {
+        const int tensor = ch / PER_T;
+        const int rem = ch - tensor * PER_T;
+        const int r = rem / CH, c16 = rem - r * CH;
+        const int j = s_idx[tile * kKeyTile + r];
+        const uint16_t* base = tensor ? a.V : a.K;
+        const uint16_t* src = base + (kv_base + (j >= 0 ? j : 0)) * D + c16 * 8;
+        cp_async16(stage + tensor * SparseSmem<D>::kTileBytes + tile_chunk_offset(r, c16), src, j >= 0 ? 16u : 0u);
+    }
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const SparseArgs a) {
+    using L = SparseSmem<D>;
+    constexpr int KW = kKeyTile / kSparseWarps;  // 16 keys per warp per tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    int* s_idx = reinterpret_cast<int*>(smem + L::kIdxOff);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x;
+    const int row = blockIdx.y;  // (b*Hkv + h)*T + t
+    const int t = row % a.T, bh = row / a.T;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    int pos = a.pos[b * a.T + t];
+    if (pos < 0 || pos >= a.N) {
+        if (tid == 0) set_status(a.status, HS2_DEV_BAD_POS);
+        pos = pos < 0 ? 0 : a.N - 1;
+    }
+    int n = a.cnt[row];
+    n = n < 0 ? 0 : (n > a.kw ? a.kw : n);
+    const int lo = split * a.C4;
+    const int nk = min(lo + a.C4, n) - lo;
+    const int64_t rows_q = static_cast<int64_t>(a.B) * a.Hq * a.T;
+    auto row_q = [&](int r) -> int { return r < a.G ? (b * a.Hq + h * a.G + r) * a.T + t : -1; };
+    const PartialRef out{a.part_ml + split * rows_q, a.part_acc + split * rows_q * D};
+
+    if (nk <= 0) {  // empty split: m = -inf, l = 0, O = 0
+        for (int e = tid; e < a.G * D; e += kSparseThreads) {
+            const int r = e / D, dc = e % D;
+            out.acc[static_cast<int64_t>(row_q(r)) * D + dc] = 0.f;
+            if (dc == 0) out.ml[row_q(r)] = make_float2(-INFINITY, 0.f);
+        }
+        return;
+    }
+
+    const int ntl = (nk + kKeyTile - 1) / kKeyTile;
+    bool bad = false;
+    for (int i = tid; i < ntl * kKeyTile; i += kSparseThreads) {
+        int j = -1;
+        if (i < nk) {
+            j = a.idx[static_cast<int64_t>(row) * a.kw + lo + i];
+            if (j < 0 || j > pos) {
+                bad = true;
+                j = -1;
+            }
+        }
+        s_idx[i] = j;
+    }
+    if (__syncthreads_or(bad) && tid == 0) set_status(a.status, HS2_DEV_BAD_INDEX);
+
+    const int64_t kv_base = static_cast<int64_t>(bh) * a.N;
+    gather_tile<D>(a, s_idx, 0, smem, kv_base);
+    cp_async_commit();
+
+    const int g = lane >> 2, c = lane & 3;
+    QTile<D> q;
+    {
+        const int r0 = row_q(g), r1 = row_q(g + 8);
+        q.load(a.Q, r0 >= 0 ? static_cast<int64_t>(r0) * D : -1, r1 >= 0 ? static_cast<int64_t>(r1) * D : -1);
+    }
+    OnlineSoftmax<D> st;
+    st.init();
+    const int key0 = warp * KW;
+    for (int i = 0; i < ntl; ++i) {
+        if (i + 1 < ntl) {
+            gather_tile<D>(a, s_idx, i + 1, smem + ((i + 1) & 1) * L::kStageBytes, kv_base);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const uint32_t kbase = smem_u32(smem + (i & 1) * L::kStageBytes);
+        const uint32_t vbase = kbase + L::kTileBytes;
+        float sc[KW / 8][4];
+        qk_tile<D, KW>(q, kbase, key0, sc);
+        const int slot0 = i * kKeyTile + key0 + 2 * c;
+#pragma unroll
+        for (int nn = 0; nn < KW / 8; ++nn)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool ok = s_idx[slot0 + nn * 8 + (e & 1)] >= 0;
+                sc[nn][e] = ok ? sc[nn][e] * a.scale_log2 : -INFINITY;
+            }
+        st.template update<KW>(sc, vbase, key0);
+        __syncthreads();  // the buffer is refilled by the next iteration's gather
+    }
+    st.finish_rows();
+    float* red = reinterpret_cast<float*>(smem);
+    stash_state<D, kSparseWarps>(st, warp, red);
+    __syncthreads();
+    merge_states<D, kSparseWarps>(red, tid, kSparseThreads, out, row_q);
+}
+
+cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st) {
+    dim3 grid(p.S4, static_cast<unsigned>(p.rows_kv));
+    if (p.d == 128) {
+        const int bytes = SparseSmem<128>::bytes(p.C4);
+        cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        sparse_attn_kernel<128><<<grid, kSparseThreads, bytes, st>>>(a);
+    } else {
+        const int bytes = SparseSmem<64>::bytes(p.C4);
+        cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        sparse_attn_kernel<64><<<grid, kSparseThreads, bytes, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace hs2

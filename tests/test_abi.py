@@ -1,0 +1,116 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry point, and
+rejects bad arguments with the documented status before launching anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from long_context_sparse_hs2_b200 import build as hs2_build
+from long_context_sparse_hs2_b200 import hs2
+from tests import parity
+from tests.oracle_pins import hand8_inputs
+import oracle.hs2_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "hs2.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    hs2_build.build()
+    return hs2.lib()
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    return re.findall(r"HS2_API\s+[\w\s\*]+?\b(hs2_\w+)\s*\(", text)
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_entry_points()
+    assert set(names) == set(hs2.ENTRY_POINTS)
+    for n in names:
+        assert getattr(L, n) is not None
+
+
+def test_version_and_status_strings(L):
+    assert hs2.version() == "1.0"
+    for s in range(6):
+        assert isinstance(hs2.status_string(s), str) and hs2.status_string(s)
+
+
+def _dims(**kw):
+    base = dict(B=1, Hq=8, Hkv=1, T=1, N=4096, d=128, k=64, W=64)
+    base.update(kw)
+    return hs2.make_dims(**base)
+
+
+def test_workspace_size(L):
+    ok = hs2.workspace_size(_dims())
+    assert ok > 0 and ok % 256 == 0
+    assert hs2.workspace_size(_dims(N=8192)) > ok
+    for bad in (dict(d=96), dict(Hq=12, Hkv=4), dict(Hq=7, Hkv=2), dict(T=0), dict(N=0), dict(k=-1),
+                dict(W=-1), dict(T=5000), dict(B=0)):
+        assert hs2.workspace_size(_dims(**bad)) == 0, bad
+    assert L.hs2_workspace_size(None) == 0
+
+
+FAKE = 1 << 20  # a 256-byte-aligned non-null address; never dereferenced (checks fail first)
+
+
+def _full(L, dims, q=FAKE, k=FAKE, v=FAKE, pos=FAKE, o=FAKE, lse=FAKE, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = hs2.workspace_size(dims)
+    return L.hs2_full_attn(ctypes.byref(dims), q, k, v, pos, o, lse, ws, ws_bytes, None)
+
+
+def test_rejects_bad_arguments_without_launching(L):
+    d = _dims()
+    assert _full(L, d, q=None) == hs2.HS2_ERR_INVALID_ARG
+    assert _full(L, d, pos=None) == hs2.HS2_ERR_INVALID_ARG
+    assert _full(L, d, k=FAKE + 8) == hs2.HS2_ERR_INVALID_ARG          # misaligned bf16 pointer
+    assert _full(L, d, lse=FAKE + 2) == hs2.HS2_ERR_INVALID_ARG        # misaligned fp32 pointer
+    assert _full(L, d, ws=None) == hs2.HS2_ERR_WORKSPACE
+    assert _full(L, d, ws=FAKE + 16) == hs2.HS2_ERR_WORKSPACE          # ws must be 256-byte aligned
+    assert _full(L, d, ws_bytes=hs2.workspace_size(d) - 1) == hs2.HS2_ERR_WORKSPACE
+    assert _full(L, _dims(d=96)) == hs2.HS2_ERR_UNSUPPORTED
+    assert _full(L, _dims(Hq=24, Hkv=8)) == hs2.HS2_ERR_UNSUPPORTED   # G = 3
+    assert _full(L, _dims(Hq=7, Hkv=2)) == hs2.HS2_ERR_INVALID_ARG
+    assert _full(L, _dims(T=4097, N=4096)) == hs2.HS2_ERR_INVALID_ARG
+    assert L.hs2_full_attn(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == hs2.HS2_ERR_INVALID_ARG
+    n = hs2.workspace_size(d)
+    assert L.hs2_select(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, n, None) == hs2.HS2_ERR_INVALID_ARG
+    assert L.hs2_sparse_attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, n, None) \
+        == hs2.HS2_ERR_INVALID_ARG
+    assert L.hs2_step(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                      n - 256, None) == hs2.HS2_ERR_WORKSPACE
+    bits = ctypes.c_uint32()
+    assert L.hs2_read_device_status(None, None, ctypes.byref(bits)) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
+    pos = torch.zeros(1, 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        hs2.step(x, x, kv, kv, pos, k=1, W=1)
+
+
+def test_selection_checker_accepts_oracle_and_rejects_wrong_sets():
+    inp = hand8_inputs()
+    r = O.step_rows(inp)[(0, 0, 1)]
+    kw = inp.k + inp.W
+    good = np.full(kw, -1)
+    good[:4] = [7, 1, 6, 4]
+    parity.check_selection(good, 4, r)
+    swapped = good.copy()
+    swapped[1] = 5   # 5 ties 1 exactly, so swapping them is allowed
+    parity.check_selection(swapped, 4, r)
+    for bad, cnt in (([7, 0, 6, 4], 4), ([7, 1, 6, 6], 4), ([7, 1, 6, -1], 3), ([1, 4, 6, 5], 4)):
+        row = np.full(kw, -1)
+        row[:len(bad)] = bad
+        with pytest.raises(AssertionError):
+            parity.check_selection(row, cnt, r)
