@@ -1,0 +1,378 @@
+"""Benchmark of the HySparse2 hybrid sparse attention step on B200.
+
+One step = one hs2_step call (full attention -> GQA-max log-softmax score -> top-k +
+window -> sparse attention with KV Reuse) over one batch of the chosen workload.  The
+default workload is the long-context decode at N = 128K (B=1, Hq=64, Hkv=8, d=128,
+T=1, k=4096, W=512), the configuration the sparse-attention queries/s and HBM GB/s
+metric is quoted on.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--impl reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload on its own
+GPU (the step has no cross-GPU exchange); timing is the max over ranks.  Prints one JSON
+line on rank 0.  ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn queries/s and achieved HBM GB/s (% of 8 TB/s) at N=128K, 1xB200"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload(name):
+    from long_context_sparse_hs2_b200.inputs import WORKLOADS
+
+    return WORKLOADS[name]
+
+
+def byte_model(w):
+    """Algorithmic bytes per step.
+
+    literal: K read once + the gathered K/V rows of the selection (the metric's formula);
+    minimum: K and V read once + gathered rows + Q in, O/LSE/idx out.
+    kv_once: K and V read once -- the algorithmic bytes of the full-attention kernel."""
+    B, Hq, Hkv, d, N, T, k, W = w.B, w.Hq, w.Hkv, w.d, w.N, w.T, w.k, w.W
+    kv_row = d * 2
+    k_bytes = B * Hkv * N * kv_row
+    sel = 0
+    for t in range(T):
+        pos = N - T + t
+        sel += min(k, max(0, pos - W + 1)) + min(W, pos + 1)
+    gathered = B * Hkv * sel * 2 * kv_row
+    q_o = B * Hq * T * d * 2 * 4 + B * Hq * T * 4 * 2 + B * Hkv * T * (k + W + 1) * 4
+    return dict(literal=k_bytes + gathered, minimum=2 * k_bytes + gathered + q_o, kv_once=2 * k_bytes,
+                gathered=gathered)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+
+def oracle_rows(w):
+    from long_context_sparse_hs2_b200.inputs import generate
+
+    inp = generate(w)
+    rows = [(b, h, t) for t in range(w.T) for b in range(w.B) for h in range(w.Hkv)]
+    return inp, rows
+
+
+def oracle_time(w, budget_s, inp_rows=None):
+    """Time the fp64 oracle on a bounded sample of the workload's selection rows."""
+    import oracle.hs2_oracle as O
+
+    inp, rows = inp_rows or oracle_rows(w)
+    done, t0 = 0, time.perf_counter()
+    for r in rows:
+        O.step_rows(inp, [r])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    per_row = el / done
+    queries_per_s = 1.0 / (per_row * w.B * w.Hkv)   # one query = all B*Hkv rows of one t
+    sample = f"{done} of {len(rows)} (b, kv head, t) rows of the '{w.name}' workload, full step per row"
+    return queries_per_s, el, sample
+
+
+def oracle_steps(w, steps, warmup):
+    """Reference arm: each step runs the oracle on one (b, kv head, t) row (cycling)."""
+    import oracle.hs2_oracle as O
+
+    inp, rows = oracle_rows(w)
+    for i in range(warmup):
+        O.step_rows(inp, [rows[i % len(rows)]])
+    t0 = time.perf_counter()
+    for i in range(steps):
+        O.step_rows(inp, [rows[(warmup + i) % len(rows)]])
+    el = time.perf_counter() - t0
+    queries = steps / (w.B * w.Hkv)
+    sample = (f"{steps} timed steps, each one (b, kv head, t) row of the '{w.name}' workload "
+              f"(1/{w.B * w.Hkv} of a query), after {warmup} warm-up rows")
+    return queries / el, el, sample
+
+
+def max_over_ranks(x, dist, device=None):
+    """Max of a float over all ranks (the slowest rank sets the step time); identity without dist."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(n_ranks, queries_per_replica_step, steps, max_ms):
+    """Whole-job queries/s: every rank ran `steps` replica steps; time is the max over ranks."""
+    return n_ranks * queries_per_replica_step * steps / (max_ms / 1000.0)
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank, dist):
+    import numpy as np
+    import torch
+    from long_context_sparse_hs2_b200 import build, hs2
+    from long_context_sparse_hs2_b200.inputs import generate
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(args.workload)
+    inp = generate(w)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    Qf, Qs, K, V = to_dev(inp.Qf), to_dev(inp.Qs), to_dev(inp.K), to_dev(inp.V)
+    pos = torch.from_numpy(inp.pos).to(dev)
+    dims = hs2.dims_of(Qf, K, w.k, w.W)
+    ws = hs2.alloc_workspace(dims, dev)
+    out = hs2.alloc_step_outputs(dims, dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def one_step():
+        hs2.step(Qf, Qs, K, V, pos, k=w.k, W=w.W, out=out, ws=ws, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def timed(n):
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            one_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return e0.elapsed_time(e1)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    torch.cuda.synchronize(dev)
+    assert hs2.read_device_status(ws, stream) == 0, "device status bits set during warm-up"
+
+    # main timed region (headline number), clocks sampled meanwhile
+    l0 = hs2.launch_count()
+    with ClockSampler(local_rank) as clk:
+        ms = timed(args.steps)
+    launches = hs2.launch_count() - l0
+    clocks = clk.summary()
+
+    # traced timed region: per-kernel CUDA-event durations on the launch stream
+    hs2.trace_enable(True)
+    ms_traced = timed(args.steps)
+    kern = hs2.trace_collect()
+    hs2.trace_enable(False)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    host_in = {n: t.cpu().pin_memory() for n, t in (("Qf", Qf), ("Qs", Qs), ("K", K), ("V", V), ("pos", pos))}
+    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in out.as_dict().items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def e2e_step():
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        hs2.step(dev_in["Qf"], dev_in["Qs"], dev_in["K"], dev_in["V"], dev_in["pos"], k=w.k, W=w.W, out=out,
+                 ws=ws, stream=stream)
+        for n, t in out.as_dict().items():
+            host_out[n].copy_(t, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms_e2e = e0.elapsed_time(e1)
+
+    ms = max_over_ranks(ms, dist, dev)
+    ms_e2e = max_over_ranks(ms_e2e, dist, dev)
+    assert hs2.read_device_status(ws, stream) == 0, "device status bits set during the timed region"
+    return dict(w=w, ms=ms, ms_traced=ms_traced, ms_e2e=ms_e2e, kern=kern, launches=launches, clocks=clocks,
+                h2d=h2d, d2h=d2h, dims=dims)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workload(args.workload)
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "T": w.T, "k": w.k,
+           "W": w.W, "global_batch": w.B * w.T * max(world, args.gpus), "seq_len": w.N,
+           "parallelism": f"replicas x{max(world, args.gpus)}",
+           "l2": "no flush: K and V (%d MiB) exceed the 126 MB L2" % (2 * w.B * w.Hkv * w.N * w.d * 2 >> 20)}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        qps, el, sample = oracle_steps(w, args.steps, args.warmup)
+        line = {"impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": cfg,
+                "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores(), "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_mod
+
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    try:
+        r = run_gpu(args, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    bm = byte_model(w)
+    n = max(world, 1)
+    step_s = r["ms"] / 1000.0 / args.steps
+    qps = replica_throughput(n, w.B * w.T, args.steps, r["ms"])
+    e2e_step_s = r["ms_e2e"] / 1000.0 / args.e2e_steps
+    kern = {k: {"avg_us": 1000.0 * v[0] / v[1], "launches": v[1], "share": v[0] / max(r["ms_traced"], 1e-9)}
+            for k, v in r["kern"].items()}
+    top = max((k for k in kern if k.startswith("full_attn")), key=lambda k: kern[k]["avg_us"], default=None)
+    roof = None
+    if top is not None:
+        achieved = bm["kv_once"] / (kern[top]["avg_us"] * 1e-6) / 1e9
+        roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": bm["kv_once"]}
+    line = {
+        "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_s * 1000.0, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q/K/V, needles, AR(1) drift)",
+        "config": cfg,
+        "hbm": {"literal_bytes_per_step": bm["literal"], "literal_gbs": bm["literal"] / step_s / 1e9,
+                "literal_frac_of_8tbs": bm["literal"] / step_s / 1e9 / NOMINAL_HBM_GBS,
+                "min_bytes_per_step": bm["minimum"], "min_gbs": bm["minimum"] / step_s / 1e9,
+                "min_frac_of_8tbs": bm["minimum"] / step_s / 1e9 / NOMINAL_HBM_GBS,
+                "min_frac_of_measured": bm["minimum"] / step_s / 1e9 / peaks["hbm_gbs"]},
+        "roofline": roof,
+        "kernels": kern,
+        "traced_ms_per_step": r["ms_traced"] / args.steps,
+        "e2e": {"value": replica_throughput(n, w.B * w.T, args.e2e_steps, r["ms_e2e"]), "unit": "queries/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_step_s * 1000.0, "steps": args.e2e_steps},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if not args.no_cpu_baseline and n == 1:
+        qps_cpu, el, sample = oracle_time(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": qps_cpu, "unit": "queries/s", "cores": cores(), "kind": "oracle",
+                                "sample": sample, "seconds": el}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -39,7 +39,8 @@
  *      idx                                : int32 [B][Hkv][T][k + W]
  *      cnt                                : int32 [B][Hkv][T]
  *  - idx row r holds cnt[r] valid key indices followed by -1 padding.  The order of
- *    the valid entries is unspecified (attention does not depend on key order).
+ *    the valid entries is unspecified (attention does not depend on key order).  When
+ *    k + W = 0 idx has no elements and may be NULL.
  *  - ws is a device workspace of at least hs2_workspace_size(dims) bytes, 256-byte
  *    aligned, owned by the caller; its contents need no initialisation and are
  *    overwritten by every call.  The library allocates no memory of its own.
@@ -141,6 +142,22 @@ HS2_API hs2_status hs2_read_device_status(const void* ws, void* stream, uint32_t
 
 /* Static, human-readable name of a status code. */
 HS2_API const char* hs2_status_string(hs2_status status);
+
+/* Per-kernel timing (tracing).  hs2_trace_enable(1) creates a fixed pool of CUDA events
+ * (host-side driver objects; no device memory) on the current device and starts recording:
+ * every entry point then records an event on its stream when it starts and after each kernel
+ * it launches.  hs2_trace_enable(0) stops recording.  Either call clears the record.
+ * hs2_trace_collect waits for the recorded events and writes, for each kernel name seen since
+ * the last collect, its summed duration in milliseconds and its launch count (at most
+ * max_entries names; names point to static strings).  It returns the number of names, -1 on
+ * a CUDA error, or -(n + 1) if the event pool ran out (the record is then incomplete).
+ * Process-global, not thread-safe: meant for profiling and benchmark runs.  Not from the
+ * pages: tracing support of this library. */
+HS2_API hs2_status hs2_trace_enable(int enable);
+HS2_API int hs2_trace_collect(const char** names, double* total_ms, int64_t* launches, int max_entries);
+
+/* Number of CUDA kernels this library has launched in this process (tracing on or off). */
+HS2_API uint64_t hs2_launch_count(void);
 
 /* Library version, (major << 16) | minor. */
 HS2_API uint32_t hs2_version(void);

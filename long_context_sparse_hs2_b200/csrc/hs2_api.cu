@@ -41,6 +41,7 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     if (x.B < 1 || x.Hq < 1 || x.Hkv < 1 || x.T < 1 || x.N < 1 || x.k < 0 || x.W < 0) return false;
     if (x.T > x.N || x.Hq % x.Hkv != 0) return false;
     if (static_cast<int64_t>(x.k) + x.W >= (int64_t(1) << 31)) return false;
+    if (x.N > (int64_t(1) << 30)) return false;
     const int64_t rows_q = static_cast<int64_t>(x.B) * x.Hq * x.T;
     const int64_t rows_kv = static_cast<int64_t>(x.B) * x.Hkv * x.T;
     if (rows_q >= (int64_t(1) << 31) || static_cast<int64_t>(x.B) * x.Hkv >= (int64_t(1) << 31)) return false;
@@ -49,6 +50,7 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     if (x.d != 64 && x.d != 128) return false;
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return false;
     if (rows_kv > 65535) return false;  // grid.y of the per-row kernels
+    if (static_cast<int64_t>(x.k) + x.W > kMaxKW) return false;
 
     Plan& P = *p;
     P.B = x.B; P.Hq = x.Hq; P.Hkv = x.Hkv; P.T = x.T; P.N = x.N; P.d = x.d; P.k = x.k; P.W = x.W; P.G = G;
@@ -66,22 +68,26 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     const int64_t slots = (P.RT == 1 ? 2 : 1) * int64_t(kSMs);
     P.S1 = choose_splits(units, tiles, slots, 256);
 
+    // sparse attention: about one CTA per SM, each gathering C4 keys (a multiple of 64, <= 1024)
     const int64_t kw = static_cast<int64_t>(x.k) + x.W;
-    P.C4 = 1024;
-    while (P.C4 > 64 && rows_kv * ((kw + P.C4 - 1) / P.C4) < 4 * kSMs) P.C4 /= 2;
+    const int64_t s4_target = std::max<int64_t>(1, kSMs / rows_kv);
+    const int64_t c4 = ((std::max<int64_t>(1, (kw + s4_target - 1) / s4_target) + 63) / 64) * 64;
+    P.C4 = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(64, c4)));
     P.S4 = static_cast<int>(std::max<int64_t>(1, (kw + P.C4 - 1) / P.C4));
     P.cand_cap = std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
+    P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
 
     size_t off = 0;
     P.off_status = off; off += 256;
     P.off_meta = off; off = align_up(off + rows_kv * kMetaInts * 4, 256);
+    P.meta_end = off;
     P.off_hist = off; off = align_up(off + rows_kv * kHistBins * 4, 256);
     P.zero_bytes = off;
     P.off_pf_ml = off; off = align_up(off + size_t(P.S1) * rows_q * 8, 256);
     P.off_pf_acc = off; off = align_up(off + size_t(P.S1) * rows_q * x.d * 4, 256);
     P.off_ps_ml = off; off = align_up(off + size_t(P.S4) * rows_q * 8, 256);
     P.off_ps_acc = off; off = align_up(off + size_t(P.S4) * rows_q * x.d * 4, 256);
-    P.off_keys = off; off = align_up(off + size_t(rows_kv) * x.N * 4, 256);
+    P.off_keys = off; off = align_up(off + size_t(rows_kv) * P.kstride * 4, 256);
     P.off_cand = off; off = align_up(off + size_t(rows_kv) * P.cand_cap * 8, 256);
     P.off_logits = off;
     if (P.mat_logits) off = align_up(off + size_t(rows_kv) * x.N * G * 4, 256);
@@ -157,35 +163,31 @@ AttnArgs attn_args(const Plan& p, const void* Q, const int32_t* pos, const Ws& w
     return a;
 }
 
+// Full-attention sweep.  combine: merge the splits here (otherwise the score kernel does it);
+// zero_from/zero_to: workspace bytes the sweep clears for the kernels after it.
 hs2_status run_full(const Plan& p, const void* Qf, const void* K, const void* V, const int32_t* pos, void* O_full,
-                    float* LSE_full, const Ws& w, bool keep_logits, cudaStream_t st) {
+                    float* LSE_full, const Ws& w, bool keep_logits, bool combine, size_t zero_from, size_t zero_to,
+                    cudaStream_t st) {
     CUtensorMap tmK, tmV;
     if (!make_kv_map(&tmK, K, p) || !make_kv_map(&tmV, V, p)) return HS2_ERR_CUDA;
     AttnArgs a = attn_args(p, Qf, pos, w);
     a.logits = keep_logits ? w.at<float>(p.off_logits) : nullptr;
+    if (zero_to > zero_from) {
+        a.zero = w.at<uint4>(zero_from);
+        a.zero_vec = static_cast<int64_t>((zero_to - zero_from) / 16);
+    }
     HS2_TRY(launch_full_attn(p, tmK, tmV, a, st));
-    CombineArgs c{a.part_ml, a.part_acc, p.S1, p.rows_q, static_cast<uint16_t*>(O_full), LSE_full};
-    HS2_TRY(launch_combine(p.d, c, st));
+    if (combine) {
+        CombineArgs c{a.part_ml, a.part_acc, p.S1, p.rows_q, static_cast<uint16_t*>(O_full), LSE_full};
+        HS2_TRY(launch_combine(p.d, c, st));
+    }
     return HS2_OK;
 }
 
-hs2_status run_select(const Plan& p, const void* Qf, const void* K, const float* LSE_full, const int32_t* pos,
-                      int32_t* idx, int32_t* cnt, const Ws& w, bool from_logits, cudaStream_t st) {
-    unsigned* status = w.at<unsigned>(p.off_status);
-    uint32_t* keys = w.at<uint32_t>(p.off_keys);
-    if (from_logits) {
-        ScoreArgs s{w.at<float>(p.off_logits), LSE_full, pos, p.B, p.Hq, p.Hkv, p.T, p.N, p.G, p.W, keys, status};
-        HS2_TRY(launch_score_from_logits(p, s, st));
-    } else {
-        CUtensorMap tmK;
-        if (!make_kv_map(&tmK, K, p)) return HS2_ERR_CUDA;
-        AttnArgs a = attn_args(p, Qf, pos, w);
-        a.lse = LSE_full;
-        a.keys = keys;
-        HS2_TRY(launch_score_sweep(p, tmK, a, st));
-    }
+TopkArgs topk_args(const Plan& p, const int32_t* pos, int32_t* idx, int32_t* cnt, const Ws& w) {
     TopkArgs t{};
-    t.keys = keys;
+    t.keys = w.at<uint32_t>(p.off_keys);
+    t.kstride = p.kstride;
     t.pos = pos;
     t.Hkv = p.Hkv; t.T = p.T; t.N = p.N; t.k = p.k; t.W = p.W;
     t.rows = p.rows_kv;
@@ -195,8 +197,45 @@ hs2_status run_select(const Plan& p, const void* Qf, const void* K, const float*
     t.cand_cap = p.cand_cap;
     t.idx = idx;
     t.cnt = cnt;
-    t.status = status;
-    HS2_TRY(launch_topk(p, t, st));
+    t.status = w.at<unsigned>(p.off_status);
+    return t;
+}
+
+// Selection from a second K sweep (needs LSE_full): keys, histogram + threshold, select.
+hs2_status run_select_sweep(const Plan& p, const void* Qf, const void* K, const float* LSE_full,
+                            const int32_t* pos, int32_t* idx, int32_t* cnt, const Ws& w, cudaStream_t st) {
+    CUtensorMap tmK;
+    if (!make_kv_map(&tmK, K, p)) return HS2_ERR_CUDA;
+    AttnArgs a = attn_args(p, Qf, pos, w);
+    a.lse = LSE_full;
+    a.keys = w.at<uint32_t>(p.off_keys);
+    a.kstride = p.kstride;
+    HS2_TRY(launch_score_sweep(p, tmK, a, st));
+    const TopkArgs t = topk_args(p, pos, idx, cnt, w);
+    HS2_TRY(launch_topk_hist(p, t, st));
+    HS2_TRY(launch_topk_select(p, t, st));
+    return HS2_OK;
+}
+
+// Selection from the kept logits, with the full-attention combine folded in.
+hs2_status run_select_kept(const Plan& p, const int32_t* pos, void* O_full, float* LSE_full, int32_t* idx,
+                           int32_t* cnt, const Ws& w, cudaStream_t st) {
+    ScoreArgs s{};
+    s.logits = w.at<float>(p.off_logits);
+    s.part_ml = w.at<float2>(p.off_pf_ml);
+    s.part_acc = w.at<float>(p.off_pf_acc);
+    s.S1 = p.S1;
+    s.pos = pos;
+    s.B = p.B; s.Hq = p.Hq; s.Hkv = p.Hkv; s.T = p.T; s.N = p.N; s.G = p.G; s.k = p.k; s.W = p.W;
+    s.O = static_cast<uint16_t*>(O_full);
+    s.LSE = LSE_full;
+    s.keys = w.at<uint32_t>(p.off_keys);
+    s.kstride = p.kstride;
+    s.hist = w.at<unsigned>(p.off_hist);
+    s.meta = w.at<int>(p.off_meta);
+    s.status = w.at<unsigned>(p.off_status);
+    HS2_TRY(launch_score_hist(p, s, st));
+    HS2_TRY(launch_topk_select(p, topk_args(p, pos, idx, cnt, w), st));
     return HS2_OK;
 }
 
@@ -215,15 +254,18 @@ hs2_status run_sparse(const Plan& p, const void* Qs, const void* K, const void* 
     s.scale_log2 = scale_log2(p);
     s.part_ml = w.at<float2>(p.off_ps_ml);
     s.part_acc = w.at<float>(p.off_ps_acc);
+    s.meta = w.at<int>(p.off_meta);
+    s.O = static_cast<uint16_t*>(O_sparse);
+    s.LSE = LSE_sparse;
     s.status = w.at<unsigned>(p.off_status);
     HS2_TRY(launch_sparse_attn(p, s, st));
-    CombineArgs c{s.part_ml, s.part_acc, p.S4, p.rows_q, static_cast<uint16_t*>(O_sparse), LSE_sparse};
-    HS2_TRY(launch_combine(p.d, c, st));
     return HS2_OK;
 }
 
 bool ok16(const void* p) { return p && aligned(p, 16); }
 bool ok4(const void* p) { return p && aligned(p, 4); }
+// idx has k + W entries per row; with k + W = 0 it is empty and may be null.
+bool ok_idx(const void* p, const Plan& P) { return (P.k + P.W == 0 && !p) || ok4(p); }
 
 }  // namespace
 }  // namespace hs2
@@ -248,8 +290,10 @@ hs2_status hs2_full_attn(const hs2_dims* dims, const void* Q_full, const void* K
     if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
+    trace_call_begin(st);
     HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));
-    return run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, false, st);
+    trace_mark("workspace_clear", st, false);
+    return run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, false, true, 0, 0, st);
 }
 
 hs2_status hs2_select(const hs2_dims* dims, const void* Q_full, const void* K, const float* LSE_full,
@@ -257,13 +301,15 @@ hs2_status hs2_select(const hs2_dims* dims, const void* Q_full, const void* K, c
     Plan p;
     hs2_status why;
     if (!make_plan(dims, &p, &why)) return why;
-    if (!ok16(Q_full) || !ok16(K) || !ok4(LSE_full) || !ok4(pos) || !ok4(idx) || !ok4(cnt))
+    if (!ok16(Q_full) || !ok16(K) || !ok4(LSE_full) || !ok4(pos) || !ok_idx(idx, p) || !ok4(cnt))
         return HS2_ERR_INVALID_ARG;
     if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
+    trace_call_begin(st);
     HS2_TRY(cudaMemsetAsync(ws, 0, p.zero_bytes, st));
-    return run_select(p, Q_full, K, LSE_full, pos, idx, cnt, w, false, st);
+    trace_mark("workspace_clear", st, false);
+    return run_select_sweep(p, Q_full, K, LSE_full, pos, idx, cnt, w, st);
 }
 
 hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, const void* K, const void* V,
@@ -272,13 +318,15 @@ hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, const voi
     Plan p;
     hs2_status why;
     if (!make_plan(dims, &p, &why)) return why;
-    if (!ok16(Q_sparse) || !ok16(K) || !ok16(V) || !ok4(pos) || !ok4(idx) || !ok4(cnt) || !ok16(O_sparse) ||
+    if (!ok16(Q_sparse) || !ok16(K) || !ok16(V) || !ok4(pos) || !ok_idx(idx, p) || !ok4(cnt) || !ok16(O_sparse) ||
         !ok4(LSE_sparse))
         return HS2_ERR_INVALID_ARG;
     if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
-    HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));
+    trace_call_begin(st);
+    HS2_TRY(cudaMemsetAsync(ws, 0, p.meta_end, st));
+    trace_mark("workspace_clear", st, false);
     return run_sparse(p, Q_sparse, K, V, pos, idx, cnt, O_sparse, LSE_sparse, w, st);
 }
 
@@ -289,15 +337,19 @@ hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_spar
     hs2_status why;
     if (!make_plan(dims, &p, &why)) return why;
     if (!ok16(Q_full) || !ok16(Q_sparse) || !ok16(K) || !ok16(V) || !ok4(pos) || !ok16(O_full) ||
-        !ok16(O_sparse) || !ok4(LSE_full) || !ok4(LSE_sparse) || !ok4(idx) || !ok4(cnt))
+        !ok16(O_sparse) || !ok4(LSE_full) || !ok4(LSE_sparse) || !ok_idx(idx, p) || !ok4(cnt))
         return HS2_ERR_INVALID_ARG;
     if (check_ws(p, ws, ws_bytes) != HS2_OK) return HS2_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
-    HS2_TRY(cudaMemsetAsync(ws, 0, p.zero_bytes, st));
-    hs2_status s = run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, p.mat_logits, st);
+    trace_call_begin(st);
+    HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));  // status word; the full sweep clears the rest
+    trace_mark("workspace_clear", st, false);
+    hs2_status s = run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, p.mat_logits, !p.mat_logits, p.off_meta,
+                            p.zero_bytes, st);
     if (s != HS2_OK) return s;
-    s = run_select(p, Q_full, K, LSE_full, pos, idx, cnt, w, p.mat_logits, st);
+    s = p.mat_logits ? run_select_kept(p, pos, O_full, LSE_full, idx, cnt, w, st)
+                     : run_select_sweep(p, Q_full, K, LSE_full, pos, idx, cnt, w, st);
     if (s != HS2_OK) return s;
     return run_sparse(p, Q_sparse, K, V, pos, idx, cnt, O_sparse, LSE_sparse, w, st);
 }

@@ -21,8 +21,14 @@ constexpr float kBinsPerUnit = 128.f;
 constexpr int kTopkChunk = 4096;     // pool keys per CTA in the histogram / emit passes
 constexpr int kMetaInts = 8;         // per-row top-k bookkeeping ints (see TopkMeta)
 
-// Per-row top-k bookkeeping in the workspace (ints; zeroed at the start of every call).
-enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDone = 2, kMetaDef = 3, kMetaCand = 4 };
+// Per-row bookkeeping in the workspace (ints; zeroed before each use, see Plan::off_meta).
+//   kMetaBin / kMetaAbove: threshold bucket of the k-th best key and the count above it
+//   kMetaDone: score/histogram CTAs finished;  kMetaDef / kMetaCand: emit counters
+//   kMetaSelDone: selection CTAs finished;     kMetaSparseDone: sparse-attention CTAs finished
+enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDone = 2, kMetaDef = 3, kMetaCand = 4, kMetaSelDone = 5,
+                kMetaSparseDone = 6 };
+constexpr int kSmemCand = 4096;      // candidates the final select keeps in shared memory
+constexpr int kMaxKW = 1 << 22;      // largest supported k + W
 
 // Everything one call needs to know about shapes, grids and workspace offsets.
 struct Plan {
@@ -37,8 +43,9 @@ struct Plan {
     int C4;             // selected keys per sparse-attention CTA
     int S4;             // sparse-attention splits per row = ceil((k+W)/C4)
     int64_t cand_cap;   // per-row capacity of the top-k candidate buffer
+    int64_t kstride;    // row stride (elements) of the score-key buffer: N rounded up to 64
     // workspace byte offsets
-    size_t off_status, off_meta, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand,
+    size_t off_status, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand,
         off_logits, zero_bytes, total;
 };
 
@@ -48,6 +55,8 @@ bool make_plan(const hs2_dims* dims, Plan* p, hs2_status* why);
 
 struct AttnArgs {
     const uint16_t* Q;     // [B][Hq][T][D]
+    uint4* zero;           // optional region the full sweep clears for the kernels after it
+    int64_t zero_vec;      // its size in 16-byte words
     const int32_t* pos;    // [B][T]
     int B, Hq, Hkv, T, N, G, W;
     int TQ, QB, S;
@@ -56,7 +65,8 @@ struct AttnArgs {
     float* part_acc;       // [S][rows_q][D]
     float* logits;         // optional [rows_kv][N][G] base-2 logits (full sweep only)
     const float* lse;      // [rows_q] natural-log LSE_full (score sweep only)
-    uint32_t* keys;        // [rows_kv][N] order-preserving score keys (score sweep only)
+    uint32_t* keys;        // [rows_kv][kstride] order-preserving score keys (score sweep only)
+    int64_t kstride;
     unsigned* status;
 };
 
@@ -72,6 +82,9 @@ struct SparseArgs {
     float scale_log2;
     float2* part_ml;       // [S4][rows_q]
     float* part_acc;       // [S4][rows_q][D]
+    int* meta;             // [rows_kv][kMetaInts] (completion counter kMetaSparseDone)
+    uint16_t* O;           // O_sparse [B][Hq][T][D]
+    float* LSE;            // LSE_sparse [B][Hq][T]
     unsigned* status;
 };
 
@@ -84,17 +97,25 @@ struct CombineArgs {
     float* LSE;            // [rows] natural log
 };
 
-struct ScoreArgs {         // scores from kept logits
-    const float* logits;   // [rows_kv][N][G]
-    const float* lse;      // [rows_q] natural log
+struct ScoreArgs {         // scores + histogram from kept logits, with the full-attention combine
+    const float* logits;   // [rows_kv][N][G] base-2 logits
+    const float2* part_ml; // full-attention split partials [S1][rows_q]
+    const float* part_acc; // [S1][rows_q][D]
+    int S1;
     const int32_t* pos;
-    int B, Hq, Hkv, T, N, G, W;
-    uint32_t* keys;        // [rows_kv][N]
+    int B, Hq, Hkv, T, N, G, k, W;
+    uint16_t* O;           // O_full [B][Hq][T][D]
+    float* LSE;            // LSE_full [B][Hq][T]
+    uint32_t* keys;        // [rows_kv][kstride]
+    int64_t kstride;
+    unsigned* hist;        // [rows_kv][kHistBins]
+    int* meta;             // [rows_kv][kMetaInts]
     unsigned* status;
 };
 
 struct TopkArgs {
-    const uint32_t* keys;  // [rows][N]
+    const uint32_t* keys;  // [rows][kstride]
+    int64_t kstride;
     const int32_t* pos;    // [B][T]
     int Hkv, T, N, k, W;
     int64_t rows;
@@ -107,14 +128,20 @@ struct TopkArgs {
     unsigned* status;
 };
 
+// ------------------------------------------------------------------ tracing (hs2_trace.cu)
+
+void trace_call_begin(cudaStream_t st);              // once at the start of every entry point
+void trace_mark(const char* name, cudaStream_t st, bool kernel = true);  // after every launch / memset
+
 // ------------------------------------------------------------------ launchers (return cudaGetLastError())
 
 cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                              cudaStream_t st);
 cudaError_t launch_score_sweep(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st);
-cudaError_t launch_score_from_logits(const Plan& p, const ScoreArgs& a, cudaStream_t st);
+cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st);
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st);
-cudaError_t launch_topk(const Plan& p, const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st);
 
 }  // namespace hs2

@@ -16,11 +16,12 @@
 // kv head: the GQA-max log-softmax selection score (in base-2 units), written as an
 // order-preserving uint32 key for every pool key j <= pos - W.
 //
-// score_from_logits_kernel: the same score from kept logits.
-// combine_kernel: split partials -> bf16 O and natural-log LSE.
+// combine_kernel: split partials -> bf16 O and natural-log LSE (used when the combine is not
+// fused into the next kernel).
 #include <algorithm>
 
 #include "attn_core.cuh"
+#include "combine.cuh"
 #include "hs2_internal.h"
 
 namespace hs2 {
@@ -111,6 +112,11 @@ __global__ void __launch_bounds__((NC + 1) * 32)
     const int bh = unit / a.QB, qb = unit % a.QB;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
 
+    if (a.zero) {  // clear the next kernels' per-row counters and histograms, spread over all CTAs
+        const int64_t cta = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+        const int64_t nthr = static_cast<int64_t>(gridDim.x) * gridDim.y * blockDim.x;
+        for (int64_t i = cta * blockDim.x + tid; i < a.zero_vec; i += nthr) a.zero[i] = make_uint4(0, 0, 0, 0);
+    }
     for (int r = tid; r < 16 * RT; r += blockDim.x) {
         const int tq = r / a.G, t = qb * a.TQ + tq;
         s_pos[r] = (tq < a.TQ && t < a.T) ? clamp_pos(a.pos[b * a.T + t], a.N, a.status) : -1;
@@ -287,8 +293,8 @@ __global__ void __launch_bounds__((NC + 1) * 32)
         const bool writer_hi = writer_lo && a.G < 16;  // with G = 16 rows g and g+8 share a query
         uint32_t* key_lo = nullptr;
         uint32_t* key_hi = nullptr;
-        if (rq_lo >= 0) key_lo = a.keys + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_lo / a.G) * a.N;
-        if (rq_hi >= 0) key_hi = a.keys + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_hi / a.G) * a.N;
+        if (rq_lo >= 0) key_lo = a.keys + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_lo / a.G) * a.kstride;
+        if (rq_hi >= 0) key_hi = a.keys + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_hi / a.G) * a.kstride;
         const int key0 = ks * KW;
         bool nonfinite = false;
         for (int i = 0; i < nt; ++i) {
@@ -316,12 +322,12 @@ __global__ void __launch_bounds__((NC + 1) * 32)
                 for (int off = 4; off < 32; off <<= 1) {
                     if (off < 4 * gl) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) sc[n][e] = fmaxf(sc[n][e], __shfl_xor_sync(0xffffffffu, sc[n][e], off));
+                        for (int e = 0; e < 4; ++e) sc[n][e] = nan_max(sc[n][e], __shfl_xor_sync(0xffffffffu, sc[n][e], off));
                     }
                 }
                 if (a.G >= 16) {
-                    sc[n][0] = fmaxf(sc[n][0], sc[n][2]);
-                    sc[n][1] = fmaxf(sc[n][1], sc[n][3]);
+                    sc[n][0] = nan_max(sc[n][0], sc[n][2]);
+                    sc[n][1] = nan_max(sc[n][1], sc[n][3]);
                 }
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -340,86 +346,15 @@ __global__ void __launch_bounds__((NC + 1) * 32)
     __syncthreads();
 }
 
-// ====================================================================== scores from kept logits
-
-template <int G>
-__global__ void __launch_bounds__(256) score_from_logits_kernel(const ScoreArgs a) {
-    const int row = blockIdx.y;  // (b*Hkv + h)*T + t
-    const int t = row % a.T, bh = row / a.T;
-    const int b = bh / a.Hkv, h = bh % a.Hkv;
-    int p = a.pos[b * a.T + t];
-    p = p < 0 ? 0 : (p >= a.N ? a.N - 1 : p);
-    const int P = p - a.W + 1;  // pool size (may be <= 0)
-    __shared__ float s_lse[G];
-    if (threadIdx.x < G) s_lse[threadIdx.x] = a.lse[(b * a.Hq + h * G + threadIdx.x) * a.T + t] * kLog2e;
-    __syncthreads();
-    const int j = blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= P) return;
-    const float* lg = a.logits + (static_cast<int64_t>(row) * a.N + j) * G;
-    float v[G];
-    if constexpr (G % 4 == 0) {
-#pragma unroll
-        for (int q = 0; q < G / 4; ++q) {
-            const float4 f = __ldcs(reinterpret_cast<const float4*>(lg) + q);
-            v[4 * q] = f.x;
-            v[4 * q + 1] = f.y;
-            v[4 * q + 2] = f.z;
-            v[4 * q + 3] = f.w;
-        }
-    } else {
-#pragma unroll
-        for (int q = 0; q < G; ++q) v[q] = lg[q];
-    }
-    float s = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < G; ++q) s = fmaxf(s, v[q] - s_lse[q]);
-    if (s != s) set_status(a.status, HS2_DEV_NONFINITE);
-    a.keys[static_cast<int64_t>(row) * a.N + j] = score_key(s);
-}
-
 // ====================================================================== combine
 
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
-    constexpr int PER = D / 32;  // dims per lane
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ float wbuf[8][256];
+    const int warp = threadIdx.x >> 5;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
     if (row >= a.rows) return;
-    float M = -INFINITY;
-    for (int s = 0; s < a.S; ++s) M = fmaxf(M, a.part_ml[s * a.rows + row].x);
-    float L = 0.f, acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < a.S; ++s) {
-            const float2 ml = a.part_ml[s * a.rows + row];
-            if (ml.x == -INFINITY) continue;
-            const float f = fast_exp2(ml.x - M);
-            L += f * ml.y;
-            const float* src = a.part_acc + (s * a.rows + row) * D + lane * PER;
-            if constexpr (PER == 4) {
-                const float4 x = *reinterpret_cast<const float4*>(src);
-                acc[0] += f * x.x;
-                acc[1] += f * x.y;
-                acc[2] += f * x.z;
-                acc[3] += f * x.w;
-            } else {
-                const float2 x = *reinterpret_cast<const float2*>(src);
-                acc[0] += f * x.x;
-                acc[1] += f * x.y;
-            }
-        }
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint32_t packed[PER / 2];
-#pragma unroll
-    for (int e = 0; e < PER / 2; ++e) packed[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-    uint16_t* dst = a.O + row * D + lane * PER;
-    if constexpr (PER == 4)
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    else
-        *reinterpret_cast<uint32_t*>(dst) = packed[0];
-    if (lane == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    warp_combine_row<D>(a.part_ml, a.part_acc, a.S, a.rows, row, wbuf[warp], a.O, a.LSE);
 }
 
 // ====================================================================== launchers
@@ -442,6 +377,7 @@ cudaError_t full_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUten
     if (e != cudaSuccess) return e;
     dim3 grid(p.S1, p.B * p.Hkv * p.QB);
     kern<<<grid, (NC + 1) * 32, L::kBytes, st>>>(tmK, tmV, a);
+    trace_mark(KEEP ? "full_attn_keep_logits" : "full_attn", st);
     return cudaGetLastError();
 }
 
@@ -455,6 +391,7 @@ cudaError_t score_sweep_variant(const Plan& p, const CUtensorMap& tmK, const Att
     if (e != cudaSuccess) return e;
     dim3 grid(p.S1, p.B * p.Hkv * p.QB);
     kern<<<grid, (NC + 1) * 32, L::kBytes, st>>>(tmK, a);
+    trace_mark("score_sweep", st);
     return cudaGetLastError();
 }
 
@@ -482,25 +419,13 @@ cudaError_t launch_score_sweep(const Plan& p, const CUtensorMap& tmK, const Attn
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_score_from_logits(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
-    dim3 grid((p.N + 255) / 256, static_cast<unsigned>(p.rows_kv));
-    switch (p.G) {
-        case 1: score_from_logits_kernel<1><<<grid, 256, 0, st>>>(a); break;
-        case 2: score_from_logits_kernel<2><<<grid, 256, 0, st>>>(a); break;
-        case 4: score_from_logits_kernel<4><<<grid, 256, 0, st>>>(a); break;
-        case 8: score_from_logits_kernel<8><<<grid, 256, 0, st>>>(a); break;
-        case 16: score_from_logits_kernel<16><<<grid, 256, 0, st>>>(a); break;
-        default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
-}
-
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st) {
     const unsigned blocks = static_cast<unsigned>((a.rows + 7) / 8);
     if (d == 128)
         combine_kernel<128><<<blocks, 256, 0, st>>>(a);
     else
         combine_kernel<64><<<blocks, 256, 0, st>>>(a);
+    trace_mark("combine", st);
     return cudaGetLastError();
 }
 

@@ -11,10 +11,12 @@
 //
 // Grid: (S4 splits, B*Hkv*T rows).  A CTA reads its C4 slots of the row's index list,
 // validates them (0 <= j <= pos; others are skipped and flagged), gathers the rows with
-// 16-byte cp.async into the same 128-byte-swizzled tile layout the TMA path uses,
-// double-buffered 64 keys at a time, and runs the shared warp attention core.  Splits
-// merge in combine_kernel.
+// 16-byte cp.async into the same 128-byte-swizzled tile layout the TMA path uses -- up to
+// four 64-key tiles in flight -- and runs the shared warp attention core.  The row's last
+// CTA to finish (a completion counter; nothing waits) merges the S4 split partials into
+// O_sparse and LSE_sparse.
 #include "attn_core.cuh"
+#include "combine.cuh"
 #include "hs2_internal.h"
 
 namespace hs2 {
@@ -24,14 +26,25 @@ namespace {
 constexpr int kSparseWarps = 4;
 constexpr int kSparseThreads = kSparseWarps * 32;
 
+constexpr int kSparseStages = 4;
+
 template <int D>
 struct SparseSmem {
     static constexpr int kTileBytes = kKeyTile * D * 2;
     static constexpr int kStageBytes = 2 * kTileBytes;  // K + V
-    static constexpr int kRingBytes = 2 * kStageBytes;
+    static constexpr int kRingBytes = kSparseStages * kStageBytes;
     static constexpr int kIdxOff = kRingBytes;
-    static constexpr int bytes(int C4) { return kIdxOff + (C4 + kKeyTile) * 4 + 1024; }
+    static constexpr int bytes(int C4) { return kIdxOff + (C4 + kKeyTile) * 4 + 16 + 1024; }
 };
+
+__device__ __forceinline__ void cp_async_wait_upto(int pending) {
+    switch (pending) {
+        case 0: cp_async_wait<0>(); break;
+        case 1: cp_async_wait<1>(); break;
+        case 2: cp_async_wait<2>(); break;
+        default: cp_async_wait<3>(); break;
+    }
+}
 
 template <int D>
 __device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_idx, int tile, uint8_t* stage,
@@ -47,6 +60,29 @@ __device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_id
         const uint16_t* src = base + (kv_base + (j >= 0 ? j : 0)) * D + c16 * 8;
         cp_async16(stage + tensor * SparseSmem<D>::kTileBytes + tile_chunk_offset(r, c16), src, j >= 0 ? 16u : 0u);
     }
+}
+
+__device__ __forceinline__ int64_t out_rows_q_base(const SparseArgs& a, int b, int h, int t) {
+    return (static_cast<int64_t>(b) * a.Hq + h * a.G) * a.T + t;  // row of head g is base + g*T
+}
+
+// The row's last split CTA merges all S4 partials of the row's G heads (one warp per head).
+template <int D>
+__device__ __forceinline__ void finish_row(const SparseArgs& a, int row, int64_t rq_base, uint8_t* smem) {
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&a.meta[static_cast<int64_t>(row) * kMetaInts + kMetaSparseDone], 1) ==
+                                    a.S4 - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int warp = threadIdx.x >> 5;
+    const int64_t rows_q = static_cast<int64_t>(a.B) * a.Hq * a.T;
+    float* wbuf = reinterpret_cast<float*>(smem) + warp * a.S4;
+    for (int g = warp; g < a.G; g += kSparseWarps)
+        warp_combine_row<D>(a.part_ml, a.part_acc, a.S4, rows_q, rq_base + static_cast<int64_t>(g) * a.T, wbuf, a.O,
+                            a.LSE);
 }
 
 }  // namespace
@@ -83,6 +119,7 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
             out.acc[static_cast<int64_t>(row_q(r)) * D + dc] = 0.f;
             if (dc == 0) out.ml[row_q(r)] = make_float2(-INFINITY, 0.f);
         }
+        finish_row<D>(a, row, out_rows_q_base(a, b, h, t), smem);
         return;
     }
 
@@ -102,8 +139,11 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     if (__syncthreads_or(bad) && tid == 0) set_status(a.status, HS2_DEV_BAD_INDEX);
 
     const int64_t kv_base = static_cast<int64_t>(bh) * a.N;
-    gather_tile<D>(a, s_idx, 0, smem, kv_base);
-    cp_async_commit();
+    const int prime = min(ntl, kSparseStages);
+    for (int i = 0; i < prime; ++i) {
+        gather_tile<D>(a, s_idx, i, smem + i * L::kStageBytes, kv_base);
+        cp_async_commit();
+    }
 
     const int g = lane >> 2, c = lane & 3;
     QTile<D> q;
@@ -115,15 +155,10 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     st.init();
     const int key0 = warp * KW;
     for (int i = 0; i < ntl; ++i) {
-        if (i + 1 < ntl) {
-            gather_tile<D>(a, s_idx, i + 1, smem + ((i + 1) & 1) * L::kStageBytes, kv_base);
-            cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
+        cp_async_wait_upto(min(ntl, i + kSparseStages) - (i + 1));  // tile i has landed
         __syncthreads();
-        const uint32_t kbase = smem_u32(smem + (i & 1) * L::kStageBytes);
+        const int stage = i % kSparseStages;
+        const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes);
         const uint32_t vbase = kbase + L::kTileBytes;
         float sc[KW / 8][4];
         qk_tile<D, KW>(q, kbase, key0, sc);
@@ -136,13 +171,18 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
                 sc[nn][e] = ok ? sc[nn][e] * a.scale_log2 : -INFINITY;
             }
         st.template update<KW>(sc, vbase, key0);
-        __syncthreads();  // the buffer is refilled by the next iteration's gather
+        __syncthreads();  // everyone is done with this stage before it is refilled
+        if (i + kSparseStages < ntl) {
+            gather_tile<D>(a, s_idx, i + kSparseStages, smem + stage * L::kStageBytes, kv_base);
+            cp_async_commit();
+        }
     }
     st.finish_rows();
     float* red = reinterpret_cast<float*>(smem);
     stash_state<D, kSparseWarps>(st, warp, red);
     __syncthreads();
     merge_states<D, kSparseWarps>(red, tid, kSparseThreads, out, row_q);
+    finish_row<D>(a, row, out_rows_q_base(a, b, h, t), smem);
 }
 
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st) {
@@ -158,6 +198,7 @@ cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t 
         if (e != cudaSuccess) return e;
         sparse_attn_kernel<64><<<grid, kSparseThreads, bytes, st>>>(a);
     }
+    trace_mark("sparse_attn_combine", st);
     return cudaGetLastError();
 }
 

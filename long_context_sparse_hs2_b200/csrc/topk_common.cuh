@@ -1,0 +1,129 @@
+// Pieces of the exact token-level top-k shared by the scoring and selection kernels.
+//
+// Keys: the fp32 score s (base-2 units) maps to an order-preserving uint32 (score_key).
+// Buckets: score_bin is a monotone, non-increasing function of the score with 1/128 of a
+// base-2 unit per bin (bin 0 = best, NaN last), so every key in a better bucket than the
+// bucket holding the k-th best key is selected outright.  Composite: (key << 32) |
+// (2^32 - 1 - j) is distinct per key and orders by (score desc, index asc) -- exactly the
+// selection rule with ties to the lower index.
+#pragma once
+
+#include "hs2_device.cuh"
+
+namespace hs2 {
+
+__device__ __forceinline__ int score_bin(uint32_t key) {
+    if (key == 0u) return kHistBins - 1;  // NaN ranks last
+    const float x = -key_score(key) * kBinsPerUnit;
+    if (!(x > 0.f)) return 0;
+    if (x >= static_cast<float>(kHistBins - 1)) return kHistBins - 1;
+    return static_cast<int>(x);
+}
+
+__device__ __forceinline__ unsigned long long composite(uint32_t key, int j) {
+    return (static_cast<unsigned long long>(key) << 32) |
+           static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(j));
+}
+__device__ __forceinline__ int composite_index(unsigned long long c) {
+    return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(c & 0xFFFFFFFFull));
+}
+
+struct RowInfo {
+    int pos;   // query position (clamped into [0, N))
+    int P;     // pool size: keys 0 .. pos-W
+    int keff;  // min(k, P) keys come from the pool
+    int wcnt;  // min(W, pos+1) window keys
+};
+
+__device__ __forceinline__ RowInfo make_row_info(const int32_t* pos, int64_t row, int Hkv, int T, int N, int k,
+                                                 int W) {
+    const int t = static_cast<int>(row % T);
+    const int b = static_cast<int>(row / (static_cast<int64_t>(Hkv) * T));
+    int p = pos[b * T + t];
+    p = p < 0 ? 0 : (p >= N ? N - 1 : p);
+    RowInfo r;
+    r.pos = p;
+    r.P = max(0, p - W + 1);
+    r.keff = min(k, r.P);
+    r.wcnt = min(W, p + 1);
+    return r;
+}
+
+// Appends the lanes with pred set to a global list; returns the lane's slot (or -1).
+__device__ __forceinline__ int warp_append(bool pred, int* counter) {
+    const unsigned mask = __ballot_sync(0xffffffffu, pred);
+    if (mask == 0u) return -1;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(mask) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(counter, __popc(mask));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    return pred ? base + __popc(mask & ((1u << lane) - 1u)) : -1;
+}
+
+// Exclusive block-wide prefix sum of one value per thread (blockDim.x a multiple of 32).
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned w = lane < nw ? s_warp[lane] : 0u;
+        unsigned wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nw) s_warp[lane] = wi - w;
+    }
+    __syncthreads();
+    const unsigned r = s_warp[warp] + incl - v;
+    __syncthreads();
+    return r;
+}
+
+// Adds this CTA's shared-memory histogram to the row's global one; the last of the row's
+// `participants` CTAs (a completion counter -- nothing waits) then finds the bucket b1 of the
+// keff-th best key and the number of keys above it, and stores them in meta.
+// blockDim.x must be 256.
+__device__ __forceinline__ void hist_flush_and_threshold(const unsigned* sh, unsigned* hist, int* meta,
+                                                         int participants, int keff, unsigned* s_warp,
+                                                         int* s_last) {
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+        if (sh[i]) atomicAdd(&hist[i], sh[i]);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *s_last = (atomicAdd(&meta[kMetaDone], 1) == participants - 1);
+    __syncthreads();
+    if (!*s_last) return;
+    __threadfence();
+    constexpr int PER = kHistBins / 256;
+    unsigned vals[PER];
+    unsigned sum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        vals[i] = __ldcg(&hist[threadIdx.x * PER + i]);
+        sum += vals[i];
+    }
+    const unsigned excl = block_exclusive_scan(sum, s_warp);
+    const unsigned need = static_cast<unsigned>(keff);
+    if (excl < need && need <= excl + sum) {
+        unsigned cum = excl;
+        for (int i = 0; i < PER; ++i) {
+            if (cum + vals[i] >= need) {
+                meta[kMetaBin] = threadIdx.x * PER + i;
+                meta[kMetaAbove] = static_cast<int>(cum);
+                break;
+            }
+            cum += vals[i];
+        }
+    }
+}
+
+}  // namespace hs2

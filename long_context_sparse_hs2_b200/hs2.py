@@ -25,7 +25,8 @@ HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUD
 DEV_BAD_POS, DEV_BAD_INDEX, DEV_NONFINITE, DEV_TIMEOUT, DEV_CAND_OVERFLOW = 0x1, 0x2, 0x4, 0x8, 0x10
 
 ENTRY_POINTS = ("hs2_workspace_size", "hs2_full_attn", "hs2_select", "hs2_sparse_attn", "hs2_step",
-                "hs2_read_device_status", "hs2_status_string", "hs2_version")
+                "hs2_read_device_status", "hs2_status_string", "hs2_trace_enable", "hs2_trace_collect",
+                "hs2_launch_count", "hs2_version")
 
 
 class Dims(ctypes.Structure):
@@ -66,6 +67,12 @@ def lib() -> ctypes.CDLL:
     L.hs2_status_string.argtypes = [ctypes.c_int]
     L.hs2_status_string.restype = ctypes.c_char_p
     L.hs2_version.restype = ctypes.c_uint32
+    L.hs2_trace_enable.argtypes = [ctypes.c_int]
+    L.hs2_trace_enable.restype = ctypes.c_int
+    L.hs2_trace_collect.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+    L.hs2_trace_collect.restype = ctypes.c_int
+    L.hs2_launch_count.restype = ctypes.c_uint64
     for f in ("hs2_full_attn", "hs2_select", "hs2_sparse_attn", "hs2_step", "hs2_read_device_status"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
@@ -234,6 +241,29 @@ def read_device_status(ws: torch.Tensor, stream=None) -> int:
     if st not in (HS2_OK, HS2_ERR_DEVICE):
         raise HS2Error(st, "hs2_read_device_status")
     return int(bits.value)
+
+
+def trace_enable(enable: bool = True) -> None:
+    """Start (or stop) per-kernel CUDA-event timing inside the library; clears the record."""
+    _check(lib().hs2_trace_enable(1 if enable else 0), "hs2_trace_enable")
+
+
+def trace_collect(max_entries: int = 64) -> Dict[str, tuple]:
+    """{kernel name: (total ms, launches)} since the last collect (waits for the events)."""
+    names = (ctypes.c_char_p * max_entries)()
+    ms = (ctypes.c_double * max_entries)()
+    cnt = (ctypes.c_int64 * max_entries)()
+    n = lib().hs2_trace_collect(names, ms, cnt, max_entries)
+    if n == -1:
+        raise HS2Error(HS2_ERR_CUDA, "hs2_trace_collect")
+    if n < 0:
+        raise RuntimeError("trace event pool exhausted: collect more often")
+    return {names[i].decode(): (ms[i], int(cnt[i])) for i in range(n)}
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(lib().hs2_launch_count())
 
 
 def version() -> str:
