@@ -128,7 +128,11 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, c
                            void* ws, size_t ws_bytes, void* stream);
 
 /* The whole hybrid step: hs2_full_attn, hs2_select and hs2_sparse_attn in order on one
- * stream, sharing intermediates through ws (when T*G <= 16 the full-attention pass
+ * stream, sharing intermediates through ws.  With one query per batch row (T = 1) and the
+ * environment variable HS2_FUSED_DECODE=1 the step runs as a single cooperative kernel when
+ * its grid fits on the device (same results up to rounding order; the workspace size depends
+ * on the setting, so query hs2_workspace_size under the same environment); when T*G <= 16 the
+ * full-attention pass
  * also keeps its logits so the selection does not read K a second time). */
 HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
                     const void* K, const void* V, const int32_t* pos,

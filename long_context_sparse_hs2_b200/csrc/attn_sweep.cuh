@@ -1,0 +1,214 @@
+// The full-attention sweep of one CTA, shared by the standalone full-attention kernel and
+// the fused decode-step kernel (sm_100a).
+//
+// Split-K flash-decode: a CTA owns one row block (the G query heads of one kv head for TQ
+// consecutive queries = 16*RT MMA rows) and one contiguous range of 64-key tiles.  A
+// producer warp streams K and V tiles into a STAGES-deep shared-memory ring with TMA (3-D
+// tensor map, 128-byte swizzle, no multicast), signalled through mbarriers with bounded
+// waits; NC consumer warps compute QK^T and PV with bf16 mma.sync and keep an online softmax
+// in base-2 units.  Each CTA writes one split partial (m, l, O) per row; the partials merge
+// with the log-sum-exp correction ("Simplified Sparse Attention via Gist Tokens", section
+// 3.6, "three-kernel split-K sparse flash-decode").  With KEEP_LOGITS the sweep also stores
+// every visible base-2 logit, [row][key][head], so the selection score can be formed
+// without reading K a second time.
+#pragma once
+
+#include "attn_core.cuh"
+
+namespace hs2 {
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ int clamp_pos(int p, int N, unsigned* status) {
+    if (p < 0 || p >= N) {
+        if (status) {
+            pdl_wait();  // the status word is cleared by the call's first kernel
+            set_status(status, HS2_DEV_BAD_POS);
+        }
+        p = p < 0 ? 0 : N - 1;
+    }
+    return p;
+}
+
+// Shared-memory layout of the streaming kernels (after 1 KB alignment).
+template <int D, int STAGES, int TENSORS>
+struct StreamSmem {
+    static constexpr int kTileBytes = kKeyTile * D * 2;                 // one tensor, one tile
+    static constexpr int kStageBytes = TENSORS * kTileBytes;
+    static constexpr int kRingBytes = STAGES * kStageBytes;
+    static constexpr int kBarOff = kRingBytes;                           // full[STAGES], empty[STAGES]
+    static constexpr int kMiscOff = kBarOff + 2 * STAGES * 8;            // abort flag + row positions
+    static constexpr int kBytes = kMiscOff + 16 + 128 * 4 + 1024;        // + alignment slack
+};
+
+// Producer side of the TMA ring: stream tiles [t_begin, t_begin + nt) of kv slice bh.
+template <int D, int STAGES, int TENSORS>
+__device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* ring, uint64_t* full,
+                              uint64_t* empty, volatile int* abort_flag, int t_begin, int nt, int bh,
+                              unsigned* status, bool stream) {
+    using L = StreamSmem<D, STAGES, TENSORS>;
+    const uint64_t pol = stream ? l2_evict_first() : l2_evict_normal();
+    prefetch_tensormap(tmK);
+    if (TENSORS == 2) prefetch_tensormap(tmV);
+    int issued = 0;
+    for (int i = 0; i < nt; ++i) {
+        const int stage = i % STAGES;
+        if (i >= STAGES && !mbar_wait(&empty[stage], ((i / STAGES) - 1) & 1, status)) {
+            *abort_flag = 1;
+            break;
+        }
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+        const int j0 = (t_begin + i) * kKeyTile;
+        uint8_t* dst = ring + stage * L::kStageBytes;
+#pragma unroll
+        for (int half = 0; half < D / 64; ++half) {
+            tma_load_3d(dst + half * (kKeyTile * 128), tmK, &full[stage], half * 64, j0, bh, pol);
+            if (TENSORS == 2)
+                tma_load_3d(dst + L::kTileBytes + half * (kKeyTile * 128), tmV, &full[stage], half * 64, j0, bh,
+                            pol);
+        }
+        ++issued;
+    }
+    // Drain: wait (bounded) for the last load issued into every stage, so no copy is still
+    // landing in shared memory when the CTA retires (matters only after an abort).
+    for (int st = 0; st < STAGES && st < issued; ++st) {
+        const int last = st + ((issued - 1 - st) / STAGES) * STAGES;
+        mbar_wait(&full[st], (last / STAGES) & 1, status);
+    }
+}
+
+
+// One CTA's share of the full-attention sweep: row block `unit`, split `split`.  Streams the
+// split's K/V tiles through the TMA ring, keeps the online softmax, optionally stores the
+// base-2 logits, and writes the split partial of every row of the block.  Returns false if a
+// pipeline wait ran out (HS2_DEV_TIMEOUT is then set).  *t_range receives the tile range.
+// Ends with the block synchronised; the ring is free again afterwards.
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS>
+__device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttnArgs& a,
+                                           uint8_t* smem, int split, int unit, int2* t_range) {
+    constexpr int NKS = NC / RT;          // warps sharing one row tile (each a key slice)
+    constexpr int KW = kKeyTile / NKS;    // keys per warp per tile
+    static_assert(NC % RT == 0 && KW % 16 == 0, "bad warp split");
+    using L = StreamSmem<D, STAGES, 2>;
+    uint8_t* ring = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* empty = full + STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff);
+    int* s_pos = reinterpret_cast<int*>(smem + L::kMiscOff + 16);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = unit / a.QB, qb = unit % a.QB;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    for (int r = tid; r < 16 * RT; r += blockDim.x) {
+        const int tq = r / a.G, t = qb * a.TQ + tq;
+        s_pos[r] = (tq < a.TQ && t < a.T) ? clamp_pos(a.pos[b * a.T + t], a.N, a.status) : -1;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NC);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    int jmax = -1;
+    for (int r = 0; r < 16 * RT; ++r) jmax = max(jmax, s_pos[r]);
+    const int ntiles = jmax >= 0 ? (jmax + kKeyTile) / kKeyTile : 0;
+    const int t_begin = static_cast<int>((static_cast<int64_t>(split) * ntiles) / a.S);
+    const int t_end = static_cast<int>((static_cast<int64_t>(split + 1) * ntiles) / a.S);
+    const int nt = t_end - t_begin;
+    *t_range = make_int2(t_begin, t_end);
+
+    OnlineSoftmax<D> st;
+    st.init();
+    const int rt = warp % RT, ks = warp / RT;
+    const int g = lane >> 2, c = lane & 3;
+    const int r_lo = rt * 16 + g, r_hi = r_lo + 8;
+    auto row_q = [&](int r) -> int {  // global query-head row of local row r, or -1
+        const int tq = r / a.G, t = qb * a.TQ + tq;
+        if (tq >= a.TQ || t >= a.T) return -1;
+        return (b * a.Hq + h * a.G + (r % a.G)) * a.T + t;
+    };
+
+    if (warp == NC) {
+        if (lane == 0)
+            produce_tiles<D, STAGES, 2>(tmK, tmV, ring, full, empty, abort_flag, t_begin, nt, bh, a.status,
+                                        a.stream_kv != 0);
+        __syncwarp();
+    } else {
+        QTile<D> q;
+        const int rq_lo = row_q(r_lo), rq_hi = row_q(r_hi);
+        q.load(a.Q, rq_lo >= 0 ? static_cast<int64_t>(rq_lo) * D : -1, rq_hi >= 0 ? static_cast<int64_t>(rq_hi) * D : -1);
+        const int p_lo = s_pos[r_lo], p_hi = s_pos[r_hi];
+        const int key0 = ks * KW;
+        float* lg_lo = nullptr;
+        float* lg_hi = nullptr;
+        const uint64_t keep = l2_evict_last();
+        if (KEEP_LOGITS) {
+            // [row_kv][N][G]: row_kv = (b*Hkv + h)*T + t
+            if (p_lo >= 0)
+                lg_lo = a.logits + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_lo / a.G) * a.N * a.G + (r_lo % a.G);
+            if (p_hi >= 0)
+                lg_hi = a.logits + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_hi / a.G) * a.N * a.G + (r_hi % a.G);
+        }
+        for (int i = 0; i < nt; ++i) {
+            const int stage = i % STAGES;
+            if (!mbar_wait(&full[stage], (i / STAGES) & 1, a.status)) {
+                *abort_flag = 1;
+                break;
+            }
+            if (*abort_flag) break;
+            const uint32_t kbase = smem_u32(ring + stage * L::kStageBytes);
+            const uint32_t vbase = kbase + L::kTileBytes;
+            float sc[KW / 8][4];
+            qk_tile<D, KW>(q, kbase, key0, sc);
+            const int jb = (t_begin + i) * kKeyTile + key0 + 2 * c;
+#pragma unroll
+            for (int n = 0; n < KW / 8; ++n) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = jb + n * 8 + (e & 1);
+                    const int p = (e < 2) ? p_lo : p_hi;
+                    const float v = sc[n][e] * a.scale_log2;
+                    sc[n][e] = (j <= p) ? v : -INFINITY;
+                    if (KEEP_LOGITS && j <= p) {
+                        float* lg = (e < 2) ? lg_lo : lg_hi;
+                        st_f32_policy(lg + static_cast<int64_t>(j) * a.G, v, keep);
+                    }
+                }
+            }
+            st.template update<KW>(sc, vbase, key0);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+        }
+        st.finish_rows();
+    }
+    __syncthreads();
+    if (*abort_flag) return false;
+
+    const PartialRef out{a.part_ml + static_cast<int64_t>(split) * (a.B * a.Hq * a.T),
+                         a.part_acc + static_cast<int64_t>(split) * (a.B * a.Hq * a.T) * D};
+    if (NKS == 1) {
+        if (warp < NC) store_partial<D>(st, out, [&](int r) { return row_q(rt * 16 + r); });
+    } else {
+        float* red = reinterpret_cast<float*>(ring);  // the ring is idle now
+        if (warp < NC) stash_state<D, NKS>(st, ks, red + rt * merge_floats<D, NKS>());
+        __syncthreads();
+        // threads of the CTA split evenly over the RT tiles
+        const int per = blockDim.x / RT;
+        const int my_rt = tid / per;
+        if (my_rt < RT)
+            merge_states<D, NKS>(red + my_rt * merge_floats<D, NKS>(), tid - my_rt * per, per, out,
+                                 [&](int r) { return row_q(my_rt * 16 + r); });
+    }
+    __syncthreads();
+    return true;
+}
+
+
+}  // namespace hs2

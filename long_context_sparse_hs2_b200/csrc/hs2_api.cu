@@ -2,6 +2,7 @@
 // plan (grids, split factors, workspace layout), TMA descriptors and launch order.
 // Declared and documented in include/hs2.h.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -66,7 +67,18 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     if (units > 65535) return false;  // grid.y of the streaming kernels
     const int64_t tiles = (x.N + kKeyTile - 1) / kKeyTile;
     const int64_t slots = (P.RT == 1 ? 2 : 1) * int64_t(kSMs);
-    P.S1 = choose_splits(units, tiles, slots, 256);
+    // The fused decode step needs every CTA resident at once: keep its grid within one wave.
+    const char* want_fused_shape = std::getenv("HS2_FUSED_DECODE");
+    const bool fused_shape = want_fused_shape && want_fused_shape[0] == '1' && x.T == 1 && P.mat_logits && units <= slots;
+    P.S1 = choose_splits(units, tiles, slots, fused_shape ? static_cast<int>(std::min<int64_t>(256, slots / units)) : 256);
+    // One decode query per batch row: the whole step can run as one kernel whose S1 x (B*Hkv)
+    // CTAs are co-resident (two per SM).
+    // The single-kernel decode step is opt-in (HS2_FUSED_DECODE=1): on B200 the kernel chain
+    // with programmatic dependent launch is faster for the benchmark shapes.
+    const char* want_fused = std::getenv("HS2_FUSED_DECODE");
+    P.fused = want_fused && want_fused[0] == '1' && x.T == 1 && P.mat_logits && units * P.S1 <= slots &&
+              ((tiles + P.S1 - 1) / P.S1) * kKeyTile <= kFusedMaxKeys &&
+              (static_cast<int64_t>(x.k) + x.W + P.S1 - 1) / P.S1 <= kFusedMaxSlice;
 
     // sparse attention: about one CTA per SM, each gathering C4 keys (a multiple of 64, <= 1024)
     const int64_t kw = static_cast<int64_t>(x.k) + x.W;
@@ -74,7 +86,8 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     const int64_t c4 = ((std::max<int64_t>(1, (kw + s4_target - 1) / s4_target) + 63) / 64) * 64;
     P.C4 = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(64, c4)));
     P.S4 = static_cast<int>(std::max<int64_t>(1, (kw + P.C4 - 1) / P.C4));
-    P.cand_cap = std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
+    P.cand_cap = P.fused ? x.N : std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
+    const int64_t sparse_slots = std::max<int64_t>(P.S4, P.fused ? P.S1 : 0);
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
 
     size_t off = 0;
@@ -85,8 +98,8 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     P.zero_bytes = off;
     P.off_pf_ml = off; off = align_up(off + size_t(P.S1) * rows_q * 8, 256);
     P.off_pf_acc = off; off = align_up(off + size_t(P.S1) * rows_q * x.d * 4, 256);
-    P.off_ps_ml = off; off = align_up(off + size_t(P.S4) * rows_q * 8, 256);
-    P.off_ps_acc = off; off = align_up(off + size_t(P.S4) * rows_q * x.d * 4, 256);
+    P.off_ps_ml = off; off = align_up(off + size_t(sparse_slots) * rows_q * 8, 256);
+    P.off_ps_acc = off; off = align_up(off + size_t(sparse_slots) * rows_q * x.d * 4, 256);
     P.off_keys = off; off = align_up(off + size_t(rows_kv) * P.kstride * 4, 256);
     P.off_cand = off; off = align_up(off + size_t(rows_kv) * P.cand_cap * 8, 256);
     P.off_logits = off;
@@ -157,6 +170,7 @@ AttnArgs attn_args(const Plan& p, const void* Q, const int32_t* pos, const Ws& w
     a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.T = p.T; a.N = p.N; a.G = p.G; a.W = p.W;
     a.TQ = p.TQ; a.QB = p.QB; a.S = p.S1;
     a.scale_log2 = scale_log2(p);
+    a.stream_kv = p.QB == 1 ? 1 : 0;  // one row block per kv head: each K/V tile is read once
     a.part_ml = w.at<float2>(p.off_pf_ml);
     a.part_acc = w.at<float>(p.off_pf_acc);
     a.status = w.at<unsigned>(p.off_status);
@@ -262,6 +276,38 @@ hs2_status run_sparse(const Plan& p, const void* Qs, const void* K, const void* 
     return HS2_OK;
 }
 
+// The fused single-kernel decode step (T = 1).  Returns HS2_ERR_UNSUPPORTED (nothing launched)
+// if the grid cannot be co-resident on this device.
+hs2_status run_fused(const Plan& p, const void* Qf, const void* Qs, const void* K, const void* V, const int32_t* pos,
+                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt,
+                     const Ws& w, cudaStream_t st) {
+    CUtensorMap tmK, tmV;
+    if (!make_kv_map(&tmK, K, p) || !make_kv_map(&tmV, V, p)) return HS2_ERR_CUDA;
+    DecodeArgs d{};
+    d.attn = attn_args(p, Qf, pos, w);
+    d.attn.logits = w.at<float>(p.off_logits);
+    d.Qs = static_cast<const uint16_t*>(Qs);
+    d.K = static_cast<const uint16_t*>(K);
+    d.V = static_cast<const uint16_t*>(V);
+    d.k = p.k;
+    d.W = p.W;
+    d.ps_ml = w.at<float2>(p.off_ps_ml);
+    d.ps_acc = w.at<float>(p.off_ps_acc);
+    d.hist = w.at<unsigned>(p.off_hist);
+    d.meta = w.at<int>(p.off_meta);
+    d.cand = w.at<unsigned long long>(p.off_cand);
+    d.cand_cap = p.cand_cap;
+    d.idx = idx;
+    d.cnt = cnt;
+    d.O_full = static_cast<uint16_t*>(O_full);
+    d.LSE_full = LSE_full;
+    d.O_sparse = static_cast<uint16_t*>(O_sparse);
+    d.LSE_sparse = LSE_sparse;
+    const cudaError_t e = launch_decode_step(p, tmK, tmV, d, st);
+    if (e == cudaErrorCooperativeLaunchTooLarge) return HS2_ERR_UNSUPPORTED;
+    return cuda_status(e);
+}
+
 bool ok16(const void* p) { return p && aligned(p, 16); }
 bool ok4(const void* p) { return p && aligned(p, 4); }
 // idx has k + W entries per row; with k + W = 0 it is empty and may be null.
@@ -291,8 +337,7 @@ hs2_status hs2_full_attn(const hs2_dims* dims, const void* Q_full, const void* K
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));
-    trace_mark("workspace_clear", st, false);
+    HS2_TRY(launch_init(ws, 256, st));
     return run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, false, true, 0, 0, st);
 }
 
@@ -307,8 +352,7 @@ hs2_status hs2_select(const hs2_dims* dims, const void* Q_full, const void* K, c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(cudaMemsetAsync(ws, 0, p.zero_bytes, st));
-    trace_mark("workspace_clear", st, false);
+    HS2_TRY(launch_init(ws, p.zero_bytes, st));
     return run_select_sweep(p, Q_full, K, LSE_full, pos, idx, cnt, w, st);
 }
 
@@ -325,8 +369,7 @@ hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, const voi
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(cudaMemsetAsync(ws, 0, p.meta_end, st));
-    trace_mark("workspace_clear", st, false);
+    HS2_TRY(launch_init(ws, p.meta_end, st));
     return run_sparse(p, Q_sparse, K, V, pos, idx, cnt, O_sparse, LSE_sparse, w, st);
 }
 
@@ -343,8 +386,15 @@ hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_spar
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(cudaMemsetAsync(ws, 0, 256, st));  // status word; the full sweep clears the rest
-    trace_mark("workspace_clear", st, false);
+    if (p.fused) {
+        HS2_TRY(launch_init(ws, p.zero_bytes, st));  // status word, per-row counters, histograms
+        const hs2_status f = run_fused(p, Q_full, Q_sparse, K, V, pos, O_full, O_sparse, LSE_full, LSE_sparse, idx,
+                                       cnt, w, st);
+        if (f != HS2_ERR_UNSUPPORTED) return f;
+        // not co-resident on this device: run the multi-kernel path below
+    } else {
+        HS2_TRY(launch_init(ws, 256, st));  // status word; the full sweep clears the rest
+    }
     hs2_status s = run_full(p, Q_full, K, V, pos, O_full, LSE_full, w, p.mat_logits, !p.mat_logits, p.off_meta,
                             p.zero_bytes, st);
     if (s != HS2_OK) return s;

@@ -27,6 +27,17 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+//
+// Kernels of one call are launched with programmatic stream serialisation: a kernel may start
+// while its predecessor drains, runs its prologue, and calls pdl_wait() before it touches
+// anything the predecessor writes (pdl_wait returns once the predecessor has completed and its
+// memory is visible; without the launch attribute it returns at once).  pdl_trigger() lets the
+// next kernel launch as soon as every CTA of this one has started.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ shared memory
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -73,22 +84,88 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (global_ns() - t0 > kWaitLimitNs) {
+            pdl_wait();  // the status word is cleared by the call's first kernel
             set_status(status, HS2_DEV_TIMEOUT);
             return false;
         }
     }
 }
 
+// ------------------------------------------------------------------ inter-CTA barrier (co-resident CTAs only)
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Barrier among the CTAs that share `ctr` (a counter cleared before the launch): each CTA adds
+// one and waits until the counter reaches `target` (= the number of barriers passed so far
+// times the number of participating CTAs).  Only for CTAs guaranteed to be co-resident
+// (cooperative launch).  The wait is bounded by kWaitLimitNs; on expiry it flags
+// HS2_DEV_TIMEOUT and returns false.  Writes made before the barrier are visible after it.
+__device__ __forceinline__ bool cta_barrier(unsigned* ctr, unsigned target, unsigned* status, int* s_flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // release: this CTA's earlier writes are visible before the count; no round trip
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+        int ok = 1;
+        if (ld_acquire(ctr) < target) {
+            const uint64_t t0 = global_ns();
+            while (ld_acquire(ctr) < target) {
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    set_status(status, HS2_DEV_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        __threadfence();  // acquire side: the other CTAs' writes are visible to the whole CTA
+        *s_flag = ok;
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+// ------------------------------------------------------------------ L2 cache policies
+
+// A stream read once (the K/V sweep) is loaded evict-first; short-lived intermediates the next
+// phase reads back (kept logits, split partials) are stored evict-last, and dropped from L2
+// with discard once consumed so they are never written back to HBM.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void st_f32_policy(float* p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+// Invalidates (without write-back) the 128-byte L2 line holding p: its data becomes undefined.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 // ------------------------------------------------------------------ TMA (no multicast)
 
-// 3-D tiled bulk tensor load global -> shared, completing on an mbarrier.
-// Coordinates are (c0 = innermost element, c1, c2).  c0 must be a multiple of 8 for bf16.
+// 3-D tiled bulk tensor load global -> shared, completing on an mbarrier, with an L2 cache
+// policy.  Coordinates are (c0 = innermost element, c1, c2).  c0 must be a multiple of 8 for bf16.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0,
-                                            int c1, int c2) {
+                                            int c1, int c2, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 

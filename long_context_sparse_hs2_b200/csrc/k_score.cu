@@ -34,25 +34,29 @@ __global__ void __launch_bounds__(256) score_hist_kernel(const ScoreArgs a) {
     const int64_t rows_q = static_cast<int64_t>(a.B) * a.Hq * a.T;
     auto row_q = [&](int g) -> int64_t { return (static_cast<int64_t>(b) * a.Hq + h * G + g) * a.T + t; };
     const int nscore = (a.N + kTopkChunk - 1) / kTopkChunk;
+    pdl_trigger();
 
     if (static_cast<int>(blockIdx.x) >= nscore) {
+        pdl_wait();
         const int g = (blockIdx.x - nscore) * 8 + warp;
         float* wbuf = reinterpret_cast<float*>(sh) + warp * (kHistBins / 8);
         if (g < G) warp_combine_row<D>(a.part_ml, a.part_acc, a.S1, rows_q, row_q(g), wbuf, a.O, a.LSE);
         return;
     }
 
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
+    // Every CTA waits for the full sweep (partials, kept logits, cleared histograms) before it
+    // can finish, so this kernel's completion implies the sweep's.
+    pdl_wait();
     const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
     if (ri.keff == 0 || ri.keff == ri.P) return;  // nothing to rank: the selection kernel takes all or none
     const int participants = (ri.P + kTopkChunk - 1) / kTopkChunk;
     const int chunk = blockIdx.x;
     if (chunk >= participants) return;
-
     for (int g = warp; g < G; g += 8) {
         const float2 ML = warp_row_ml(a.part_ml, a.S1, rows_q, row_q(g));
         if (lane == 0) s_lse2[g] = lse2_of(ML);
     }
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
     float lse[G];
 #pragma unroll
@@ -108,20 +112,19 @@ cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st
     const int nscore = (p.N + kTopkChunk - 1) / kTopkChunk;
     const int ncomb = (p.G + 7) / 8;
     dim3 grid(nscore + ncomb, static_cast<unsigned>(p.rows_kv));
-#define HS2_SH(G_)                                                                        \
-    case G_:                                                                              \
-        if (p.d == 128)                                                                   \
-            score_hist_kernel<G_, 128><<<grid, 256, 0, st>>>(a);                          \
-        else                                                                              \
-            score_hist_kernel<G_, 64><<<grid, 256, 0, st>>>(a);                           \
+#define HS2_SH(G_)                                                                                          \
+    case G_:                                                                                                \
+        e = p.d == 128 ? launch_pdl(score_hist_kernel<G_, 128>, grid, dim3(256), 0, st, a)                  \
+                       : launch_pdl(score_hist_kernel<G_, 64>, grid, dim3(256), 0, st, a);                  \
         break;
+    cudaError_t e = cudaErrorInvalidValue;
     switch (p.G) {
         HS2_SH(1) HS2_SH(2) HS2_SH(4) HS2_SH(8) HS2_SH(16)
         default: return cudaErrorInvalidValue;
     }
 #undef HS2_SH
     trace_mark("score_hist", st);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace hs2

@@ -100,7 +100,9 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     const int row = blockIdx.y;  // (b*Hkv + h)*T + t
     const int t = row % a.T, bh = row / a.T;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
+    pdl_trigger();
     int pos = a.pos[b * a.T + t];
+    pdl_wait();  // idx / cnt (and cleared counters) come from the kernels before
     if (pos < 0 || pos >= a.N) {
         if (tid == 0) set_status(a.status, HS2_DEV_BAD_POS);
         pos = pos < 0 ? 0 : a.N - 1;
@@ -191,15 +193,16 @@ cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t 
         const int bytes = SparseSmem<128>::bytes(p.C4);
         cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
-        sparse_attn_kernel<128><<<grid, kSparseThreads, bytes, st>>>(a);
-    } else {
-        const int bytes = SparseSmem<64>::bytes(p.C4);
-        cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e != cudaSuccess) return e;
-        sparse_attn_kernel<64><<<grid, kSparseThreads, bytes, st>>>(a);
+        e = launch_pdl(sparse_attn_kernel<128>, grid, dim3(kSparseThreads), bytes, st, a);
+        trace_mark("sparse_attn_combine", st);
+        return e;
     }
+    const int bytes = SparseSmem<64>::bytes(p.C4);
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(sparse_attn_kernel<64>, grid, dim3(kSparseThreads), bytes, st, a);
     trace_mark("sparse_attn_combine", st);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace hs2

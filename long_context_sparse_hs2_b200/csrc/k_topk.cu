@@ -28,11 +28,13 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(const TopkArgs a) {
     __shared__ unsigned s_warp[32];
     __shared__ int s_last;
     const int64_t row = blockIdx.y;
+    pdl_trigger();
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
+    pdl_wait();  // keys from the score sweep (every CTA waits before it can finish)
     const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
     if (ri.keff == 0 || ri.keff == ri.P) return;
     const int participants = (ri.P + kTopkChunk - 1) / kTopkChunk;
     if (static_cast<int>(blockIdx.x) >= participants) return;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
     const int j0 = blockIdx.x * kTopkChunk, j1 = min(j0 + kTopkChunk, ri.P);
     const uint32_t* keys = a.keys + row * a.kstride;
@@ -80,9 +82,40 @@ struct KeyScanSource {  // overflow path: every pool key of the row whose bucket
 // most significant first; stops as soon as the remaining digits are free).
 template <class Src>
 __device__ unsigned long long radix_threshold(const Src& src, unsigned need, unsigned* h, unsigned* s_small) {
-    unsigned long long prefix = 0ull;
-    const int lane = threadIdx.x & 31;
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // Bits every element shares need no pass: start at the highest digit where they differ.
+    __shared__ unsigned long long s_and[32], s_or[32];
+    unsigned long long all_and = ~0ull, any_or = 0ull;
+    for (int i = threadIdx.x; i < src.size(); i += blockDim.x) {
+        unsigned long long c;
+        if (src.get(i, c)) {
+            all_and &= c;
+            any_or |= c;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        all_and &= __shfl_xor_sync(0xffffffffu, all_and, o);
+        any_or |= __shfl_xor_sync(0xffffffffu, any_or, o);
+    }
+    if (lane == 0) {
+        s_and[warp] = all_and;
+        s_or[warp] = any_or;
+    }
+    __syncthreads();
+    all_and = ~0ull;
+    any_or = 0ull;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+        all_and &= s_and[w];
+        any_or |= s_or[w];
+    }
+    __syncthreads();
+    const unsigned long long differ = all_and ^ any_or;
+    if (differ == 0ull) return all_and;  // a single element (composites are distinct)
+    const int top = 63 - __clzll(static_cast<long long>(differ));
+    const int first_shift = (top / 8) * 8;
+    unsigned long long prefix = first_shift >= 56 ? 0ull : (all_and & (~0ull << (first_shift + 8)));
+    for (int shift = first_shift; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0u;
         if (threadIdx.x == 0) s_small[0] = s_small[1] = 0u;
         __syncthreads();
@@ -153,10 +186,14 @@ __global__ void __launch_bounds__(256) topk_select_kernel(const TopkArgs a) {
     __shared__ unsigned long long s_cand[kSmemCand];
     __shared__ unsigned h[256];
     __shared__ unsigned s_small[2];
-    __shared__ int s_count, s_last;
+    __shared__ int s_count, s_last, s_base;
+    __shared__ int s_cnt[2];
+    static_assert(kTopkChunk % (4 * 256) == 0, "whole 16-byte key loads per thread");
     const int64_t row = blockIdx.y;
     const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
     const int participants = max(1, (ri.P + kTopkChunk - 1) / kTopkChunk);
+    pdl_trigger();
+    pdl_wait();  // keys, histogram threshold and cleared counters from the kernels before
     if (static_cast<int>(blockIdx.x) >= participants) return;
     const int kw = a.k + a.W;
     int32_t* idx = a.idx + row * kw;
@@ -172,24 +209,55 @@ __global__ void __launch_bounds__(256) topk_select_kernel(const TopkArgs a) {
     } else if (ranked) {
         const uint32_t* keys = a.keys + row * a.kstride;
         unsigned long long* cand = a.cand + row * a.cand_cap;
-        // 4 consecutive keys per lane per 16-byte load; a warp covers 128 keys per step
-        for (int base = j0 + 4 * static_cast<int>(threadIdx.x & ~31u); base < j1; base += 4 * blockDim.x) {
-            const int j = base + 4 * static_cast<int>(threadIdx.x & 31);
+        // 16 keys per thread as four 16-byte loads; pass 1 counts, one global atomic per CTA
+        // reserves the CTA's slots, pass 2 writes with shared-memory slot counters.
+        constexpr int V4 = kTopkChunk / (4 * 256);
+        uint32_t kk[V4][4];
+        int bins[V4][4], ndef = 0, ncnd = 0;
+#pragma unroll
+        for (int v = 0; v < V4; ++v) {
+            const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v);
             uint4 q = make_uint4(0, 0, 0, 0);
             if (j < j1) q = __ldcs(reinterpret_cast<const uint4*>(keys + j));
-            const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+            kk[v][0] = q.x; kk[v][1] = q.y; kk[v][2] = q.z; kk[v][3] = q.w;
+        }
+#pragma unroll
+        for (int v = 0; v < V4; ++v)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const bool valid = j + e < j1;
-                const int bin = valid ? score_bin(kk[e]) : kHistBins;
-                const bool def = valid && bin < b1;
-                const bool cnd = valid && bin == b1;
-                const int sd = warp_append(def, &meta[kMetaDef]);
-                if (def && sd < above) out[sd] = j + e;
-                const int sc = warp_append(cnd, &meta[kMetaCand]);
-                if (cnd && sc < a.cand_cap) cand[sc] = composite(kk[e], j + e);
+                const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v) + e;
+                bins[v][e] = j < j1 ? score_bin(kk[v][e]) : kHistBins;
+                ndef += bins[v][e] < b1;
+                ncnd += bins[v][e] == b1;
             }
+        if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
+            ncnd += __shfl_xor_sync(0xffffffffu, ncnd, o);
         }
+        if ((threadIdx.x & 31) == 0) {
+            atomicAdd(&s_cnt[0], ndef);
+            atomicAdd(&s_cnt[1], ncnd);
+        }
+        __syncthreads();
+        const int def_base = block_reserve(s_cnt[0], &meta[kMetaDef], &s_base);
+        const int cnd_base = block_reserve(s_cnt[1], &meta[kMetaCand], &s_base);
+        if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int v = 0; v < V4; ++v)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v) + e;
+                const bool def = bins[v][e] < b1;
+                const bool cnd = bins[v][e] == b1;
+                const int sd = warp_append(def, &s_cnt[0]);
+                if (def && def_base + sd < above) out[def_base + sd] = j;
+                const int sc = warp_append(cnd, &s_cnt[1]);
+                if (cnd && cnd_base + sc < a.cand_cap) cand[cnd_base + sc] = composite(kk[v][e], j);
+            }
     }
 
     // completion: the row's last CTA finishes the row
@@ -231,16 +299,16 @@ __global__ void __launch_bounds__(256) topk_select_kernel(const TopkArgs a) {
 
 cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st) {
     dim3 grid((p.N + kTopkChunk - 1) / kTopkChunk, static_cast<unsigned>(p.rows_kv));
-    topk_hist_kernel<<<grid, 256, 0, st>>>(a);
+    const cudaError_t e = launch_pdl(topk_hist_kernel, grid, dim3(256), 0, st, a);
     trace_mark("topk_hist", st);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st) {
     dim3 grid((p.N + kTopkChunk - 1) / kTopkChunk, static_cast<unsigned>(p.rows_kv));
-    topk_select_kernel<<<grid, 256, 0, st>>>(a);
+    const cudaError_t e = launch_pdl(topk_select_kernel, grid, dim3(256), 0, st, a);
     trace_mark("topk_select", st);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace hs2

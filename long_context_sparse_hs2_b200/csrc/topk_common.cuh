@@ -1,7 +1,7 @@
 // Pieces of the exact token-level top-k shared by the scoring and selection kernels.
 //
 // Keys: the fp32 score s (base-2 units) maps to an order-preserving uint32 (score_key).
-// Buckets: score_bin is a monotone, non-increasing function of the score with 1/128 of a
+// Buckets: score_bin is a monotone, non-increasing function of the score with 1/32 of a
 // base-2 unit per bin (bin 0 = best, NaN last), so every key in a better bucket than the
 // bucket holding the k-th best key is selected outright.  Composite: (key << 32) |
 // (2^32 - 1 - j) is distinct per key and orders by (score desc, index asc) -- exactly the
@@ -59,6 +59,33 @@ __device__ __forceinline__ int warp_append(bool pred, int* counter) {
     if (lane == leader) base = atomicAdd(counter, __popc(mask));
     base = __shfl_sync(0xffffffffu, base, leader);
     return pred ? base + __popc(mask & ((1u << lane) - 1u)) : -1;
+}
+
+// Reserves `n` consecutive slots of a global list for the whole CTA with one atomic: call from
+// all threads with the CTA's total; returns the base slot (broadcast through *s_base).
+__device__ __forceinline__ int block_reserve(int n, int* counter, int* s_base) {
+    if (threadIdx.x == 0) *s_base = n > 0 ? atomicAdd(counter, n) : 0;
+    __syncthreads();
+    const int base = *s_base;
+    __syncthreads();
+    return base;
+}
+
+// Reserves n0 and n1 slots of two adjacent list counters (ctr[0], ctr[1], 8-byte aligned) with
+// one 64-bit atomic for the whole CTA; returns both bases.  Call from all threads.
+__device__ __forceinline__ int2 block_reserve2(int n0, int n1, int* ctr, unsigned long long* s_base) {
+    if (threadIdx.x == 0) {
+        const unsigned long long add = (static_cast<unsigned long long>(static_cast<unsigned>(n1)) << 32) |
+                                       static_cast<unsigned>(n0);
+        *s_base = add ? atomicAdd(reinterpret_cast<unsigned long long*>(ctr), add) : 0ull;
+        if (!add) {
+            // nothing to reserve: the bases are not needed
+        }
+    }
+    __syncthreads();
+    const unsigned long long v = *s_base;
+    __syncthreads();
+    return make_int2(static_cast<int>(v & 0xFFFFFFFFull), static_cast<int>(v >> 32));
 }
 
 // Exclusive block-wide prefix sum of one value per thread (blockDim.x a multiple of 32).

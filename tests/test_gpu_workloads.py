@@ -58,9 +58,14 @@ def check_all_rows(inp, idx, cnt):
     np.testing.assert_array_equal(np.where(wc > 0, first, 0), np.where(wc > 0, pos - wc + 1, 0))
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["chain", "fused"])
 @pytest.mark.parametrize("name", list(SAMPLES))
-def test_workload_full_size(name):
+def test_workload_full_size(name, fused, monkeypatch):
     w = WORKLOADS[name]
+    if fused:
+        if w.T != 1:
+            pytest.skip("the single-kernel step is for T = 1")
+        monkeypatch.setenv("HS2_FUSED_DECODE", "1")
     inp = generate(w)
     g = parity.gpu_inputs(inp)
     ws = hs2.alloc_workspace(hs2.dims_of(g["Q_full"], g["K"], w.k, w.W), "cuda")
