@@ -26,6 +26,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn queries/s and achieved HBM GB/s (% of 8 TB/s) at N=128K, 1xB200"
+# DRAM bytes (read + write) per launch of the roofline kernel from an ncu capture of the same
+# kernel and workload (profiles/full_attn_long_decode.md); None where no capture matches the
+# current kernel.
+NCU_TRAFFIC = {("long", "full_attn_keep_logits"): 536923392 + 6701312}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -44,6 +48,12 @@ def workload(name):
     from long_context_sparse_hs2_b200.inputs import WORKLOADS
 
     return WORKLOADS[name]
+
+
+def flop_model(w):
+    """Tensor FLOPs of the full-attention layer (QK^T and PV over every visible key)."""
+    visible = sum(w.N - w.T + t + 1 for t in range(w.T))
+    return 4.0 * w.B * w.Hq * w.d * visible
 
 
 def byte_model(w):
@@ -343,12 +353,20 @@ def main():
     top = max((k for k in kern if k.startswith("full_attn")), key=lambda k: kern[k]["avg_us"], default=None)
     roof = None
     if top is not None:
-        achieved = bm["kv_once"] / (kern[top]["avg_us"] * 1e-6) / 1e9
-        roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                else "fallback 6.65 TB/s",
-                "algorithmic_bytes_per_launch": bm["kv_once"]}
+        secs = kern[top]["avg_us"] * 1e-6
+        if w.T * (w.Hq // w.Hkv) > 16:
+            # many query rows per kv head: the full-attention pass is a dense contraction
+            achieved = flop_model(w) / secs / 1e12
+            roof = {"bound": "tensor", "kernel": top, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                    "peak_source": f"{peak_src} bf16 dense (MEASURED_PEAKS.json bf16_tflops, burst)",
+                    "algorithmic_flops_per_launch": flop_model(w)}
+        else:
+            achieved = bm["kv_once"] / secs / 1e9
+            roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((w.name, top)),
+                    "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                    "algorithmic_bytes_per_launch": bm["kv_once"]}
     line = {
         "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_s * 1000.0, "higher_is_better": True, "scaling": "weak",

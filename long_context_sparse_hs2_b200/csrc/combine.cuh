@@ -151,6 +151,51 @@ __device__ __forceinline__ void block_combine_row(const float2* __restrict__ par
     __syncthreads();
 }
 
+// The whole CTA merges the split partials of nh rows at once (the G query heads of one
+// selection row: rows row0 + g * stride).  Warps first turn each row's (m, l) into per-split
+// weights (s_w[g * S + s]); then every thread owns float4 columns (row, 4 dims) and sums its
+// splits with up to U loads in flight.  s_w: nh * S floats, s_ml: nh float2.  Call from all
+// threads (contains barriers).
+template <int D, int U = 32>
+__device__ __forceinline__ void block_combine_rows(const float2* __restrict__ part_ml,
+                                                   const float* __restrict__ part_acc, int S, int64_t rows,
+                                                   int64_t row0, int64_t stride, int nh, float* s_w, float2* s_ml,
+                                                   uint16_t* O, float* LSE) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int g = warp; g < nh; g += nw) {
+        const float2 ML = warp_row_weights(part_ml, S, rows, row0 + g * stride, s_w + g * S);
+        if (lane == 0) s_ml[g] = ML;
+    }
+    __syncthreads();
+    constexpr int C4 = D / 4;  // float4 columns per row
+    for (int col = threadIdx.x; col < nh * C4; col += blockDim.x) {
+        const int g = col / C4, c = col % C4;
+        const int64_t row = row0 + g * stride;
+        const float* src = part_acc + row * D + c * 4;
+        const float* w = s_w + g * S;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int base = 0; base < S; base += U) {
+            float4 x[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (base + u < S) x[u] = __ldcg(reinterpret_cast<const float4*>(src + (base + u) * rows * D));
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (base + u < S) {
+                    const float wt = w[base + u];
+                    acc.x += wt * x[u].x;
+                    acc.y += wt * x[u].y;
+                    acc.z += wt * x[u].z;
+                    acc.w += wt * x[u].w;
+                }
+        }
+        *reinterpret_cast<uint2*>(O + row * D + c * 4) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        if (c == 0) LSE[row] = lse2_of(s_ml[g]) * kLn2;
+    }
+    __syncthreads();
+}
+
 // NaN-propagating max (fmaxf drops NaN operands; a NaN score must stay NaN).
 __device__ __forceinline__ float nan_max(float a, float b) { return (a > b || a != a) ? a : b; }
 

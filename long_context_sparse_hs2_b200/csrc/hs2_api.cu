@@ -86,6 +86,9 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     const int64_t c4 = ((std::max<int64_t>(1, (kw + s4_target - 1) / s4_target) + 63) / 64) * 64;
     P.C4 = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(64, c4)));
     P.S4 = static_cast<int>(std::max<int64_t>(1, (kw + P.C4 - 1) / P.C4));
+    // combine scratch: the sparse combine keeps G * S4 weights in the gather ring, the score
+    // kernel's combine CTA G * S1 weights in its histogram scratch
+    if (static_cast<int64_t>(G) * P.S4 > 8192 || static_cast<int64_t>(G) * P.S1 > 4096) return false;
     P.cand_cap = P.fused ? x.N : std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
     const int64_t sparse_slots = std::max<int64_t>(P.S4, P.fused ? P.S1 : 0);
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;

@@ -22,8 +22,8 @@
 //       its definite winners, window slice and final winners, all KV Reuse index-list
 //       entries -> a sparse split partial.  No barrier is needed before it.
 //   B3  every sparse partial is written.
-//   E   CTA `split` merges the sparse partials of head `split` into O_sparse / LSE_sparse, and
-//       CTA G + `split` the full partials of head `split` into O_full / LSE_full.
+//   E   split 0 merges the sparse partials of the G heads into O_sparse / LSE_sparse and
+//       split 1 the full partials into O_full / LSE_full (each CTA-wide, all heads at once).
 //
 // Sources: token-level selection with forced recent tokens and KV Reuse ("HySparse2 od
 // Xiaomi zkracuje zpracovani dlouheho kontextu", section "Proc neni nutne znovu zpracovat
@@ -491,16 +491,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(const __grid_c
     if (!cta_barrier(bar, 4u * S, status, &s_flag)) return;  // B3: every sparse partial is written
 
     // ---------------------------------------------------------------- E: combines
-    // task g < G: O_sparse / LSE_sparse of head g; task G + g: O_full / LSE_full of head g
+    // split 0 merges the sparse partials of all G heads, split 1 (0 if S == 1) the full ones
     {
-        float* red = reinterpret_cast<float*>(smem + kFusedRingOff);  // 5 warps x D floats
-        for (int task = split; task < 2 * G; task += S) {
-            if (task < G)
-                block_combine_row<D>(a.ps_ml, a.ps_acc, S, rows_q, row_q(task), wbuf, red, a.O_sparse, a.LSE_sparse);
-            else
-                block_combine_row<D>(at.part_ml, at.part_acc, S, rows_q, row_q(task - G), wbuf, red, a.O_full,
-                                     a.LSE_full);
-        }
+        float* s_w = reinterpret_cast<float*>(smem + kFusedRingOff);
+        float2* s_ml = reinterpret_cast<float2*>(smem + kFusedRingOff + 16 * 256 * 4);
+        if (split == 0)
+            block_combine_rows<D, 16>(a.ps_ml, a.ps_acc, S, rows_q, row_q(0), 1, G, s_w, s_ml, a.O_sparse,
+                                  a.LSE_sparse);
+        if (split == (S > 1 ? 1 : 0))
+            block_combine_rows<D, 16>(at.part_ml, at.part_acc, S, rows_q, row_q(0), 1, G, s_w, s_ml, a.O_full,
+                                  a.LSE_full);
     }
 }
 

@@ -13,8 +13,8 @@
 //     the split partials, forms every key's score (base-2 units, NaN-propagating max), writes
 //     the order-preserving key, and bins it in a shared-memory histogram that is added to
 //     the row's global histogram; the row's last CTA finds the threshold bucket.
-//   x >= nscore: merges the split partials of up to 8 of the row's query heads into O_full
-//     and LSE_full (the full-attention combine, off the critical path of the scoring CTAs).
+//   x == nscore: merges the split partials of the row's G query heads into O_full and
+//     LSE_full (the full-attention combine, off the critical path of the scoring CTAs).
 #include "combine.cuh"
 #include "topk_common.cuh"
 
@@ -22,7 +22,8 @@ namespace hs2 {
 
 template <int G, int D>
 __global__ void __launch_bounds__(256) score_hist_kernel(const ScoreArgs a) {
-    __shared__ unsigned sh[kHistBins];  // histogram, or the combine CTAs' weight buffers
+    constexpr int kScratch = kHistBins > 16 * 256 + 64 ? kHistBins : 16 * 256 + 64;
+    __shared__ unsigned sh[kScratch];  // histogram, or the combine CTA's weights (G * S1 <= 4096)
     __shared__ unsigned s_warp[32];
     __shared__ int s_last;
     __shared__ float s_lse2[G];
@@ -36,11 +37,11 @@ __global__ void __launch_bounds__(256) score_hist_kernel(const ScoreArgs a) {
     const int nscore = (a.N + kTopkChunk - 1) / kTopkChunk;
     pdl_trigger();
 
-    if (static_cast<int>(blockIdx.x) >= nscore) {
+    if (static_cast<int>(blockIdx.x) >= nscore) {  // the full-attention combine of this row's G heads
         pdl_wait();
-        const int g = (blockIdx.x - nscore) * 8 + warp;
-        float* wbuf = reinterpret_cast<float*>(sh) + warp * (kHistBins / 8);
-        if (g < G) warp_combine_row<D>(a.part_ml, a.part_acc, a.S1, rows_q, row_q(g), wbuf, a.O, a.LSE);
+        float* s_w = reinterpret_cast<float*>(sh);
+        float2* s_ml = reinterpret_cast<float2*>(sh + 16 * 256);
+        block_combine_rows<D, 8>(a.part_ml, a.part_acc, a.S1, rows_q, row_q(0), a.T, G, s_w, s_ml, a.O, a.LSE);
         return;
     }
 
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(256) score_hist_kernel(const ScoreArgs a) {
 
 cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
     const int nscore = (p.N + kTopkChunk - 1) / kTopkChunk;
-    const int ncomb = (p.G + 7) / 8;
+    const int ncomb = 1;
     dim3 grid(nscore + ncomb, static_cast<unsigned>(p.rows_kv));
 #define HS2_SH(G_)                                                                                          \
     case G_:                                                                                                \

@@ -23,42 +23,48 @@ namespace hs2 {
 
 namespace {
 
-constexpr int kSparseWarps = 4;
+constexpr int kSparseWarps = 8;
 constexpr int kSparseThreads = kSparseWarps * 32;
+constexpr int kSparseTile = 2 * kKeyTile;  // keys per pipeline step: two 64-key sub-tiles
 
-constexpr int kSparseStages = 4;
+constexpr int kSparseStages = 2;
 
 template <int D>
 struct SparseSmem {
-    static constexpr int kTileBytes = kKeyTile * D * 2;
-    static constexpr int kStageBytes = 2 * kTileBytes;  // K + V
+    static constexpr int kTileBytes = kKeyTile * D * 2;    // one 64-key sub-tile of K (or V)
+    static constexpr int kSubBytes = 2 * kTileBytes;       // K + V of one sub-tile
+    static constexpr int kStageBytes = 2 * kSubBytes;      // two sub-tiles = one 128-key step
     static constexpr int kRingBytes = kSparseStages * kStageBytes;
     static constexpr int kIdxOff = kRingBytes;
-    static constexpr int bytes(int C4) { return kIdxOff + (C4 + kKeyTile) * 4 + 16 + 1024; }
+    static constexpr int bytes(int C4) { return kIdxOff + (C4 + kSparseTile) * 4 + 16 + 1024; }
 };
 
 __device__ __forceinline__ void cp_async_wait_upto(int pending) {
-    switch (pending) {
-        case 0: cp_async_wait<0>(); break;
-        case 1: cp_async_wait<1>(); break;
-        case 2: cp_async_wait<2>(); break;
-        default: cp_async_wait<3>(); break;
-    }
+    if (pending <= 0)
+        cp_async_wait<0>();
+    else
+        cp_async_wait<1>();
 }
 
+// Gathers the K and V rows of 128-key step `tile` into a stage: sub-tile u (keys 64u..64u+63
+// of the step) at u * kSubBytes, K then V, each in the swizzled 64-key tile layout.
 template <int D>
 __device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_idx, int tile, uint8_t* stage,
                                             int64_t kv_base) {
     constexpr int CH = D / 8;                 // 16-byte chunks per row
-    constexpr int PER_T = kKeyTile * CH;      // chunks per tensor per tile
-    for (int ch = threadIdx.x; ch < 2 * PER_T; ch += kSparseThreads) {
-        const int tensor = ch / PER_T;
-        const int rem = ch - tensor * PER_T;
+    constexpr int PER_T = kKeyTile * CH;      // chunks per tensor per sub-tile
+    for (int ch = threadIdx.x; ch < 4 * PER_T; ch += kSparseThreads) {
+        const int sub = ch / (2 * PER_T);
+        const int rem2 = ch - sub * 2 * PER_T;
+        const int tensor = rem2 / PER_T;
+        const int rem = rem2 - tensor * PER_T;
         const int r = rem / CH, c16 = rem - r * CH;
-        const int j = s_idx[tile * kKeyTile + r];
+        const int j = s_idx[tile * kSparseTile + sub * kKeyTile + r];
         const uint16_t* base = tensor ? a.V : a.K;
         const uint16_t* src = base + (kv_base + (j >= 0 ? j : 0)) * D + c16 * 8;
-        cp_async16(stage + tensor * SparseSmem<D>::kTileBytes + tile_chunk_offset(r, c16), src, j >= 0 ? 16u : 0u);
+        cp_async16(stage + sub * SparseSmem<D>::kSubBytes + tensor * SparseSmem<D>::kTileBytes +
+                       tile_chunk_offset(r, c16),
+                   src, j >= 0 ? 16u : 0u);
     }
 }
 
@@ -77,12 +83,10 @@ __device__ __forceinline__ void finish_row(const SparseArgs& a, int row, int64_t
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const int warp = threadIdx.x >> 5;
     const int64_t rows_q = static_cast<int64_t>(a.B) * a.Hq * a.T;
-    float* wbuf = reinterpret_cast<float*>(smem) + warp * a.S4;
-    for (int g = warp; g < a.G; g += kSparseWarps)
-        warp_combine_row<D>(a.part_ml, a.part_acc, a.S4, rows_q, rq_base + static_cast<int64_t>(g) * a.T, wbuf, a.O,
-                            a.LSE);
+    float* s_w = reinterpret_cast<float*>(smem);                       // G * S4 weights
+    float2* s_ml = reinterpret_cast<float2*>(smem) + a.G * a.S4 / 2 + 1;  // after the weights
+    block_combine_rows<D>(a.part_ml, a.part_acc, a.S4, rows_q, rq_base, a.T, a.G, s_w, s_ml, a.O, a.LSE);
 }
 
 }  // namespace
@@ -90,7 +94,7 @@ __device__ __forceinline__ void finish_row(const SparseArgs& a, int row, int64_t
 template <int D>
 __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const SparseArgs a) {
     using L = SparseSmem<D>;
-    constexpr int KW = kKeyTile / kSparseWarps;  // 16 keys per warp per tile
+    constexpr int KW = 16;  // keys per warp per step: warps 0-3 take sub-tile 0, warps 4-7 sub-tile 1
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     int* s_idx = reinterpret_cast<int*>(smem + L::kIdxOff);
@@ -125,9 +129,9 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
         return;
     }
 
-    const int ntl = (nk + kKeyTile - 1) / kKeyTile;
+    const int ntl = (nk + kSparseTile - 1) / kSparseTile;
     bool bad = false;
-    for (int i = tid; i < ntl * kKeyTile; i += kSparseThreads) {
+    for (int i = tid; i < ntl * kSparseTile; i += kSparseThreads) {
         int j = -1;
         if (i < nk) {
             j = a.idx[static_cast<int64_t>(row) * a.kw + lo + i];
@@ -155,16 +159,17 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     }
     OnlineSoftmax<D> st;
     st.init();
-    const int key0 = warp * KW;
+    const int sub = warp >> 2;
+    const int key0 = (warp & 3) * KW;
     for (int i = 0; i < ntl; ++i) {
-        cp_async_wait_upto(min(ntl, i + kSparseStages) - (i + 1));  // tile i has landed
+        cp_async_wait_upto(min(ntl, i + kSparseStages) - (i + 1));  // step i has landed
         __syncthreads();
         const int stage = i % kSparseStages;
-        const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes);
+        const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes + sub * L::kSubBytes);
         const uint32_t vbase = kbase + L::kTileBytes;
         float sc[KW / 8][4];
         qk_tile<D, KW>(q, kbase, key0, sc);
-        const int slot0 = i * kKeyTile + key0 + 2 * c;
+        const int slot0 = i * kSparseTile + sub * kKeyTile + key0 + 2 * c;
 #pragma unroll
         for (int nn = 0; nn < KW / 8; ++nn)
 #pragma unroll

@@ -186,7 +186,8 @@ __global__ void __launch_bounds__(256) topk_select_kernel(const TopkArgs a) {
     __shared__ unsigned long long s_cand[kSmemCand];
     __shared__ unsigned h[256];
     __shared__ unsigned s_small[2];
-    __shared__ int s_count, s_last, s_base;
+    __shared__ int s_count, s_last;
+    __shared__ unsigned long long s_base2;
     __shared__ int s_cnt[2];
     static_assert(kTopkChunk % (4 * 256) == 0, "whole 16-byte key loads per thread");
     const int64_t row = blockIdx.y;
@@ -242,8 +243,8 @@ __global__ void __launch_bounds__(256) topk_select_kernel(const TopkArgs a) {
             atomicAdd(&s_cnt[1], ncnd);
         }
         __syncthreads();
-        const int def_base = block_reserve(s_cnt[0], &meta[kMetaDef], &s_base);
-        const int cnd_base = block_reserve(s_cnt[1], &meta[kMetaCand], &s_base);
+        const int2 bases = block_reserve2(s_cnt[0], s_cnt[1], &meta[kMetaDef], &s_base2);
+        const int def_base = bases.x, cnd_base = bases.y;
         if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
         __syncthreads();
 #pragma unroll
