@@ -139,6 +139,34 @@ HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,
                     int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device array that hs2_sparse_attn_static uses as its scratch. */
+#define HS2_STATIC_SCRATCH_BYTES (4u << 20)
+
+/* hs2_sparse_attn without a workspace argument, for callers that cannot allocate device
+ * memory at the point of the call (an engine serving requests from fixed memory pools, a
+ * plugin inside a program that owns all device memory, a path that cannot afford an
+ * allocation or a size query per call).  The pages have no counterpart: this is a convenience
+ * of this library.  Same arguments, layouts and results as hs2_sparse_attn, minus ws/ws_bytes.
+ *
+ *  - Scratch: one file-scope device array of HS2_STATIC_SCRATCH_BYTES (4 MiB) that every GPU
+ *    loading the library holds until the process exits.  The call allocates nothing (no
+ *    cudaMalloc / cudaFree, no allocating library routine).
+ *  - Limit: shapes whose scratch (per-row counters plus split partials, about
+ *    B*Hq*T * ceil((k+W)/C) * (d+2) * 4 bytes for the library's split size C) exceeds the array
+ *    are rejected with HS2_ERR_WORKSPACE before anything is launched; decode shapes up to a
+ *    few hundred query-head rows fit.
+ *  - Set-up: the first call on each device looks up the array's device address (while that
+ *    device is current); make that first call before any stream capture.
+ *  - Sharing: every call on a device uses the same array and leaves its contents behind; each
+ *    call clears what must start at zero.  Calls whose GPU work overlaps (other streams, other
+ *    host threads) race on the array and give undefined results: serialise them.
+ *  - Device status bits go to the array's first word; hs2_read_device_status cannot reach it,
+ *    so problems are reported only through the outputs (skipped indices, clamped positions). */
+HS2_API hs2_status hs2_sparse_attn_static(const hs2_dims* dims, const void* Q_sparse, const void* K,
+                                          const void* V, const int32_t* pos, const int32_t* idx,
+                                          const int32_t* cnt, void* O_sparse, float* LSE_sparse,
+                                          void* stream);
+
 /* Copies the device status word out of ws and waits for the stream (the only synchronising
  * call).  *bits receives the HS2_DEV_* bits; returns HS2_ERR_DEVICE if any bit other than
  * HS2_DEV_CAND_OVERFLOW is set, else HS2_OK. */

@@ -26,7 +26,8 @@ DEV_BAD_POS, DEV_BAD_INDEX, DEV_NONFINITE, DEV_TIMEOUT, DEV_CAND_OVERFLOW = 0x1,
 
 ENTRY_POINTS = ("hs2_workspace_size", "hs2_full_attn", "hs2_select", "hs2_sparse_attn", "hs2_step",
                 "hs2_read_device_status", "hs2_status_string", "hs2_trace_enable", "hs2_trace_collect",
-                "hs2_launch_count", "hs2_version")
+                "hs2_launch_count", "hs2_version", "hs2_sparse_attn_static")
+STATIC_SCRATCH_BYTES = 4 << 20  # HS2_STATIC_SCRATCH_BYTES
 
 
 class Dims(ctypes.Structure):
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
     L.hs2_select.argtypes = [dp, vp, vp, f32p, i32p, i32p, i32p, vp, sz, vp]
     L.hs2_sparse_attn.argtypes = [dp, vp, vp, vp, i32p, i32p, i32p, vp, f32p, vp, sz, vp]
     L.hs2_step.argtypes = [dp, vp, vp, vp, vp, i32p, vp, vp, f32p, f32p, i32p, i32p, vp, sz, vp]
+    L.hs2_sparse_attn_static.argtypes = [dp, vp, vp, vp, i32p, i32p, i32p, vp, f32p, vp]
+    L.hs2_sparse_attn_static.restype = ctypes.c_int
     L.hs2_read_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.hs2_status_string.argtypes = [ctypes.c_int]
     L.hs2_status_string.restype = ctypes.c_char_p
@@ -188,6 +191,25 @@ def sparse_attn(Q_sparse, K, V, pos, idx, cnt, *, k: int, W: int, O_sparse=None,
     _check(lib().hs2_sparse_attn(ctypes.byref(dm), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(idx), _p(cnt),
                                  _p(O_sparse), _p(LSE_sparse), _p(ws), ws.numel(), _stream(stream)),
            "hs2_sparse_attn")
+    return O_sparse, LSE_sparse
+
+
+def sparse_attn_static(Q_sparse, K, V, pos, idx, cnt, *, k: int, W: int, O_sparse=None, LSE_sparse=None,
+                       stream=None):
+    """hs2_sparse_attn_static: the sparse layer with its scratch in the library's fixed device
+    array (no workspace).  The outputs are allocated here only if the caller passes none."""
+    dm = dims_of(Q_sparse, K, k, W)
+    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
+    _need(Q_sparse, "Q_sparse", torch.bfloat16, (B, Hq, T, d))
+    _need(K, "K", torch.bfloat16, (B, Hkv, N, d))
+    _need(V, "V", torch.bfloat16, (B, Hkv, N, d))
+    _need(pos, "pos", torch.int32, (B, T))
+    _need(idx, "idx", torch.int32, (B, Hkv, T, k + W))
+    _need(cnt, "cnt", torch.int32, (B, Hkv, T))
+    O_sparse = torch.empty_like(Q_sparse) if O_sparse is None else O_sparse
+    LSE_sparse = torch.empty((B, Hq, T), dtype=torch.float32, device=K.device) if LSE_sparse is None else LSE_sparse
+    _check(lib().hs2_sparse_attn_static(ctypes.byref(dm), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(idx), _p(cnt),
+                                        _p(O_sparse), _p(LSE_sparse), _stream(stream)), "hs2_sparse_attn_static")
     return O_sparse, LSE_sparse
 
 
