@@ -227,7 +227,8 @@ hs2_status run_select_sweep(const Plan& p, const void* Qf, const void* K, const 
     a.lse = LSE_full;
     a.keys = w.at<uint32_t>(p.off_keys);
     a.kstride = p.kstride;
-    HS2_TRY(launch_score_sweep(p, tmK, a, st));
+    a.k = p.k;
+    HS2_TRY(launch_score_sweep(p, p.S1, tmK, a, st));
     const TopkArgs t = topk_args(p, pos, idx, cnt, w);
     HS2_TRY(launch_topk_hist(p, t, st));
     HS2_TRY(launch_topk_select(p, t, st));

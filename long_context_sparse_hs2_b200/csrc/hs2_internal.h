@@ -19,7 +19,8 @@ constexpr int kSMs = 148;            // B200 streaming multiprocessors
 constexpr int kHistBins = 2048;      // top-k histogram: 1/32 of a base-2 score unit per bin
 constexpr float kBinsPerUnit = 32.f;
 constexpr int kTopkChunk = 4096;     // pool keys per CTA in the histogram / emit passes
-constexpr int kMetaInts = 8;         // per-row top-k bookkeeping ints (see TopkMeta)
+constexpr int kMetaInts = 8;
+constexpr int kSweepMaxTiles = 65535 / 64;  // tiles per score-sweep CTA (16-bit histogram counters)         // per-row top-k bookkeeping ints (see TopkMeta)
 
 // Per-row bookkeeping in the workspace (ints; zeroed before each use, see Plan::off_meta).
 //   kMetaBin / kMetaAbove: threshold bucket of the k-th best key and the count above it
@@ -71,6 +72,7 @@ struct AttnArgs {
     const float* lse;      // [rows_q] natural-log LSE_full (score sweep only)
     uint32_t* keys;        // [rows_kv][kstride] order-preserving score keys (score sweep only)
     int64_t kstride;
+    int k;
     unsigned* status;
 };
 
@@ -194,7 +196,7 @@ cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st);  // clears ws[
 
 cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                              cudaStream_t st);
-cudaError_t launch_score_sweep(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st);
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st);

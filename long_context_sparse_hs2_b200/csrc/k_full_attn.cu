@@ -13,6 +13,7 @@
 
 #include "attn_sweep.cuh"
 #include "combine.cuh"
+#include "topk_common.cuh"
 #include "hs2_internal.h"
 
 namespace hs2 {
@@ -40,6 +41,11 @@ __global__ void __launch_bounds__((NC + 1) * 32)
 }
 
 // ====================================================================== score sweep (second K pass)
+//
+// MMA row m of 16-row tile rt holds query rt*Q8 + t_in, head g, with Q8 = 16/G queries per tile
+// and, for m < 8: t_in = m % Q8, g = m / Q8; for m >= 8: the same query and head g + G/2 (G = 1:
+// query m).  A lane's two accumulator rows m and m+8 are then two heads of one query, so the max
+// over the G heads is one local max plus log2(G/2) lane shuffles (instead of log2(G)).
 
 template <int D, int RT, int NC, int STAGES>
 __global__ void __launch_bounds__((NC + 1) * 32)
@@ -53,17 +59,30 @@ __global__ void __launch_bounds__((NC + 1) * 32)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
     uint64_t* empty = full + STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff);
-    int* s_pos = reinterpret_cast<int*>(smem + L::kMiscOff + 16);
+    int* s_pos = reinterpret_cast<int*>(smem + L::kMiscOff + 16);  // per query of the block
+    __shared__ int s_row[16 * RT], s_rank[16 * RT];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, unit = blockIdx.y;
     const int bh = unit / a.QB, qb = unit % a.QB;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const int G = a.G;
+    const int Q8 = G >= 2 ? 16 / G : 16;
+    const int nq = a.TQ;  // queries in this row block (the last block may have fewer valid)
     pdl_trigger();
 
-    for (int r = tid; r < 16 * RT; r += blockDim.x) {
-        const int tq = r / a.G, t = qb * a.TQ + tq;
-        s_pos[r] = (tq < a.TQ && t < a.T) ? clamp_pos(a.pos[b * a.T + t], a.N, nullptr) : -1;
+    for (int q = tid; q < nq; q += blockDim.x) {
+        const int t = qb * a.TQ + q;
+        int p = -1, rank = 0;
+        if (t < a.T) {
+            p = clamp_pos(a.pos[b * a.T + t], a.N, nullptr);
+            const int P = max(0, p - a.W + 1);
+            const int keff = min(a.k, P);
+            rank = keff > 0 && keff < P;  // only these rows need ranked keys
+        }
+        s_pos[q] = p;
+        s_row[q] = bh * a.T + t;
+        s_rank[q] = rank;
     }
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -75,11 +94,11 @@ __global__ void __launch_bounds__((NC + 1) * 32)
     }
     __syncthreads();
 
-    // only pool keys (j <= pos - W) are scored
+    // only pool keys (j <= pos - W) of rows that need ranking are scored
     int jmax = -1;
-    for (int r = 0; r < 16 * RT; ++r)
-        if (s_pos[r] >= 0) jmax = max(jmax, s_pos[r] - a.W);
-    const int ntiles = jmax >= 0 ? (jmax + kKeyTile) / kKeyTile : 0;  // 0 when every pool is empty
+    for (int q = 0; q < nq; ++q)
+        if (s_pos[q] >= 0 && s_rank[q]) jmax = max(jmax, s_pos[q] - a.W);
+    const int ntiles = jmax >= 0 ? (jmax + kKeyTile) / kKeyTile : 0;
     const int t_begin = static_cast<int>((static_cast<int64_t>(split) * ntiles) / a.S);
     const int t_end = static_cast<int>((static_cast<int64_t>(split + 1) * ntiles) / a.S);
     const int nt = t_end - t_begin;
@@ -89,36 +108,41 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             produce_tiles<D, STAGES, 1>(&tmK, &tmK, ring, full, empty, abort_flag, t_begin, nt, bh, a.status,
                                         a.stream_kv != 0);
         __syncwarp();
+    }
+    const int rt = warp % RT, ks = warp / RT;
+    const int m_lo = lane >> 2, c = lane & 3;
+    // (query in block, head) of MMA rows m_lo and m_lo + 8 of tile rt
+    int tq_lo, g_lo, tq_hi, g_hi;
+    if (G >= 2) {
+        tq_lo = tq_hi = rt * Q8 + m_lo % Q8;
+        g_lo = m_lo / Q8;
+        g_hi = g_lo + G / 2;
     } else {
-        const int rt = warp % RT, ks = warp / RT;
-        const int g = lane >> 2, c = lane & 3;
-        const int r_lo = rt * 16 + g, r_hi = r_lo + 8;
-        auto row_q = [&](int r) -> int {
-            const int tq = r / a.G, t = qb * a.TQ + tq;
-            if (tq >= a.TQ || t >= a.T) return -1;
-            return (b * a.Hq + h * a.G + (r % a.G)) * a.T + t;
-        };
+        tq_lo = rt * 16 + m_lo;
+        tq_hi = tq_lo + 8;
+        g_lo = g_hi = 0;
+    }
+    auto row_q = [&](int tq, int gg) -> int {
+        const int t = qb * a.TQ + tq;
+        if (tq >= a.TQ || t >= a.T) return -1;
+        return (b * a.Hq + h * G + gg) * a.T + t;
+    };
+    const bool writer = G >= 2 ? (m_lo < Q8) : true;
+    bool nonfinite = false;
+    if (warp < NC) {
         QTile<D> q;
-        const int rq_lo = row_q(r_lo), rq_hi = row_q(r_hi);
+        const int rq_lo = row_q(tq_lo, g_lo), rq_hi = row_q(tq_hi, g_hi);
         q.load(a.Q, rq_lo >= 0 ? static_cast<int64_t>(rq_lo) * D : -1, rq_hi >= 0 ? static_cast<int64_t>(rq_hi) * D : -1);
         pdl_wait();  // LSE_full comes from the previous kernel
         // base-2 LSE of the two rows (+inf for padding rows so their scores are -inf)
         const float lse_lo = rq_lo >= 0 ? a.lse[rq_lo] * kLog2e : INFINITY;
         const float lse_hi = rq_hi >= 0 ? a.lse[rq_hi] * kLog2e : INFINITY;
-        // last pool key of each row's query (-1: empty pool / padding)
-        const int pl_lo = s_pos[r_lo] >= 0 ? s_pos[r_lo] - a.W : -1;
-        const int pl_hi = s_pos[r_hi] >= 0 ? s_pos[r_hi] - a.W : -1;
-        // group of G consecutive rows = one query; reduce over the lane bits that index g
-        constexpr int kMaxGroupLanes = 8;  // rows g = lane>>2 span 8 values per half
-        const int gl = a.G < kMaxGroupLanes ? a.G : kMaxGroupLanes;
-        const bool writer_lo = (g % gl) == 0;
-        const bool writer_hi = writer_lo && a.G < 16;  // with G = 16 rows g and g+8 share a query
-        uint32_t* key_lo = nullptr;
-        uint32_t* key_hi = nullptr;
-        if (rq_lo >= 0) key_lo = a.keys + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_lo / a.G) * a.kstride;
-        if (rq_hi >= 0) key_hi = a.keys + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_hi / a.G) * a.kstride;
+        // last pool key of each row's query (-1: nothing to rank)
+        const int pl_lo = (rq_lo >= 0 && s_rank[tq_lo]) ? s_pos[tq_lo] - a.W : -1;
+        const int pl_hi = (rq_hi >= 0 && s_rank[tq_hi]) ? s_pos[tq_hi] - a.W : -1;
+        uint32_t* key_lo = rq_lo >= 0 ? a.keys + static_cast<int64_t>(s_row[tq_lo]) * a.kstride : nullptr;
+        uint32_t* key_hi = rq_hi >= 0 ? a.keys + static_cast<int64_t>(s_row[tq_hi]) * a.kstride : nullptr;
         const int key0 = ks * KW;
-        bool nonfinite = false;
         for (int i = 0; i < nt; ++i) {
             const int stage = i % STAGES;
             if (!mbar_wait(&full[stage], (i / STAGES) & 1, a.status)) {
@@ -134,38 +158,38 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             const int jb = (t_begin + i) * kKeyTile + key0 + 2 * c;
 #pragma unroll
             for (int n = 0; n < KW / 8; ++n) {
+                float v[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float lse = (e < 2) ? lse_lo : lse_hi;
-                    sc[n][e] = sc[n][e] * a.scale_log2 - lse;
-                }
-                // max over the G heads of each query
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    if (off < 4 * gl) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) sc[n][e] = nan_max(sc[n][e], __shfl_xor_sync(0xffffffffu, sc[n][e], off));
+                for (int e = 0; e < 4; ++e) v[e] = sc[n][e] * a.scale_log2 - ((e < 2) ? lse_lo : lse_hi);
+                if (G >= 2) {
+                    v[0] = nan_max(v[0], v[2]);  // heads g and g + G/2 of the same query
+                    v[1] = nan_max(v[1], v[3]);
+                    for (int off = 4 * Q8; off < 32; off <<= 1) {
+                        v[0] = nan_max(v[0], __shfl_xor_sync(0xffffffffu, v[0], off));
+                        v[1] = nan_max(v[1], __shfl_xor_sync(0xffffffffu, v[1], off));
                     }
                 }
-                if (a.G >= 16) {
-                    sc[n][0] = nan_max(sc[n][0], sc[n][2]);
-                    sc[n][1] = nan_max(sc[n][1], sc[n][3]);
-                }
+                if (writer) {
+                    const int nrow = G >= 2 ? 1 : 2;
+                    for (int r = 0; r < nrow; ++r) {
+                        const int pl = r == 0 ? pl_lo : pl_hi;
+                        uint32_t* kr = r == 0 ? key_lo : key_hi;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = jb + n * 8 + (e & 1);
-                    const bool lo = e < 2;
-                    const int pl = lo ? pl_lo : pl_hi;
-                    if ((lo ? writer_lo : writer_hi) && j <= pl) {
-                        nonfinite |= (sc[n][e] != sc[n][e]);
-                        (lo ? key_lo : key_hi)[j] = score_key(sc[n][e]);
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = jb + n * 8 + e;
+                            if (j <= pl) {
+                                const float sv = v[2 * r + e];
+                                nonfinite |= (sv != sv);
+                                kr[j] = score_key(sv);
+                            }
+                        }
                     }
                 }
             }
         }
-        if (__any_sync(0xffffffffu, nonfinite) && lane == 0) set_status(a.status, HS2_DEV_NONFINITE);
     }
     __syncthreads();
+    if (__syncthreads_or(nonfinite) && tid == 0) set_status(a.status, HS2_DEV_NONFINITE);
 }
 
 // ====================================================================== combine
@@ -206,14 +230,15 @@ cudaError_t full_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUten
 }
 
 template <int D, int RT>
-cudaError_t score_sweep_variant(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st) {
+cudaError_t score_sweep_variant(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a,
+                                cudaStream_t st) {
     constexpr int NC = RT >= 8 ? 8 : 4;
     constexpr int STAGES = D == 128 ? 6 : 12;
     using L = StreamSmem<D, STAGES, 1>;
     auto kern = score_sweep_kernel<D, RT, NC, STAGES>;
     cudaError_t e = set_smem(kern, L::kBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.S1, p.B * p.Hkv * p.QB);
+    dim3 grid(splits, p.B * p.Hkv * p.QB);
     e = launch_pdl(kern, grid, dim3((NC + 1) * 32), L::kBytes, st, tmK, a);
     trace_mark("score_sweep", st);
     return e;
@@ -234,9 +259,10 @@ cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtens
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_score_sweep(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a,
+                               cudaStream_t st) {
 #define HS2_SS(D_, RT_) \
-    if (p.d == D_ && p.RT == RT_) return score_sweep_variant<D_, RT_>(p, tmK, a, st);
+    if (p.d == D_ && p.RT == RT_) return score_sweep_variant<D_, RT_>(p, splits, tmK, a, st);
     HS2_SS(64, 1) HS2_SS(64, 2) HS2_SS(64, 4) HS2_SS(64, 8)
     HS2_SS(128, 1) HS2_SS(128, 2) HS2_SS(128, 4) HS2_SS(128, 8)
 #undef HS2_SS

@@ -182,7 +182,7 @@ __device__ void emit_at_least(const Src& src, unsigned long long thr, unsigned n
 
 // ====================================================================== select: emit, then exact threshold
 
-__global__ void __launch_bounds__(256) topk_select_kernel(const TopkArgs a) {
+__global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
     __shared__ unsigned long long s_cand[kSmemCand];
     __shared__ unsigned h[256];
     __shared__ unsigned s_small[2];
