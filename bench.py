@@ -350,7 +350,8 @@ def main():
     e2e_step_s = r["ms_e2e"] / 1000.0 / args.e2e_steps
     kern = {k: {"avg_us": 1000.0 * v[0] / v[1], "launches": v[1], "share": v[0] / max(r["ms_traced"], 1e-9)}
             for k, v in r["kern"].items()}
-    top = max((k for k in kern if k.startswith("full_attn")), key=lambda k: kern[k]["avg_us"], default=None)
+    top = max((k for k in kern if k.startswith("full_attn") or k == "umma_attn"), key=lambda k: kern[k]["avg_us"],
+              default=None)
     roof = None
     if top is not None:
         secs = kern[top]["avg_us"] * 1e-6

@@ -71,6 +71,20 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     const char* want_fused_shape = std::getenv("HS2_FUSED_DECODE");
     const bool fused_shape = want_fused_shape && want_fused_shape[0] == '1' && x.T == 1 && P.mat_logits && units <= slots;
     P.S1 = choose_splits(units, tiles, slots, fused_shape ? static_cast<int>(std::min<int64_t>(256, slots / units)) : 256);
+    P.S2 = P.S1;
+    // 128-row query tiles: the full sweep runs on the tcgen05 tensor cores (HS2_UMMA=0 keeps the
+    // mma.sync sweep), one CTA per SM, two query tiles per CTA -- or one, with the key range
+    // split between the CTA's two streams, when a kv head has a single query tile.
+    const char* want_umma = std::getenv("HS2_UMMA");
+    P.umma = P.RT == 8 && !(want_umma && want_umma[0] == '0');
+    P.umma_split_keys = P.QB == 1;
+    P.SU = 1;
+    if (P.umma) {
+        const int64_t uunits = static_cast<int64_t>(x.B) * x.Hkv * (P.umma_split_keys ? P.QB : (P.QB + 1) / 2);
+        const int64_t utiles = (x.N + 127) / 128;
+        P.SU = choose_splits(uunits, utiles, kSMs, 128);
+        P.S1 = P.SU * (P.umma_split_keys ? 2 : 1);
+    }
     // One decode query per batch row: the whole step can run as one kernel whose S1 x (B*Hkv)
     // CTAs are co-resident (two per SM).
     // The single-kernel decode step is opt-in (HS2_FUSED_DECODE=1): on B200 the kernel chain
@@ -132,13 +146,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view [B*Hkv][N][d] of a K or V cache; 64 x 64 boxes, 128-byte swizzle, zero fill out of range.
-bool make_kv_map(CUtensorMap* m, const void* base, const Plan& p) {
+// 3-D view [B*Hkv][N][d] of a K or V cache; boxes of 64 dims x `rows` keys, 128-byte swizzle,
+// zero fill out of range.
+bool make_kv_map(CUtensorMap* m, const void* base, const Plan& p, int rows = kKeyTile) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {cuuint64_t(p.d), cuuint64_t(p.N), cuuint64_t(p.B) * p.Hkv};
     const cuuint64_t strides[2] = {cuuint64_t(p.d) * 2, cuuint64_t(p.N) * p.d * 2};
-    const cuuint32_t box[3] = {64, cuuint32_t(kKeyTile), 1};
+    const cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
     const cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -186,14 +201,18 @@ hs2_status run_full(const Plan& p, const void* Qf, const void* K, const void* V,
                     float* LSE_full, const Ws& w, bool keep_logits, bool combine, size_t zero_from, size_t zero_to,
                     cudaStream_t st) {
     CUtensorMap tmK, tmV;
-    if (!make_kv_map(&tmK, K, p) || !make_kv_map(&tmV, V, p)) return HS2_ERR_CUDA;
+    const int box_rows = p.umma ? 128 : kKeyTile;
+    if (!make_kv_map(&tmK, K, p, box_rows) || !make_kv_map(&tmV, V, p, box_rows)) return HS2_ERR_CUDA;
     AttnArgs a = attn_args(p, Qf, pos, w);
     a.logits = keep_logits ? w.at<float>(p.off_logits) : nullptr;
     if (zero_to > zero_from) {
         a.zero = w.at<uint4>(zero_from);
         a.zero_vec = static_cast<int64_t>((zero_to - zero_from) / 16);
     }
-    HS2_TRY(launch_full_attn(p, tmK, tmV, a, st));
+    if (p.umma)
+        HS2_TRY(launch_umma_attn(p, tmK, tmV, a, st));
+    else
+        HS2_TRY(launch_full_attn(p, tmK, tmV, a, st));
     if (combine) {
         CombineArgs c{a.part_ml, a.part_acc, p.S1, p.rows_q, static_cast<uint16_t*>(O_full), LSE_full};
         HS2_TRY(launch_combine(p.d, c, st));
@@ -228,7 +247,8 @@ hs2_status run_select_sweep(const Plan& p, const void* Qf, const void* K, const 
     a.keys = w.at<uint32_t>(p.off_keys);
     a.kstride = p.kstride;
     a.k = p.k;
-    HS2_TRY(launch_score_sweep(p, p.S1, tmK, a, st));
+    a.S = p.S2;
+    HS2_TRY(launch_score_sweep(p, p.S2, tmK, a, st));
     const TopkArgs t = topk_args(p, pos, idx, cnt, w);
     HS2_TRY(launch_topk_hist(p, t, st));
     HS2_TRY(launch_topk_select(p, t, st));

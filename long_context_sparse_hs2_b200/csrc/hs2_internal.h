@@ -41,7 +41,11 @@ struct Plan {
     int RT;             // 16-row MMA tiles per attention row block (1, 2, 4, 8)
     int TQ;             // queries per row block = 16*RT/G
     int QB;             // row blocks per (b, kv head) = ceil(T / TQ)
-    int S1;             // split-K factor of the full-attention sweep
+    int S1;             // split partials per row written by the full-attention sweep
+    int S2;             // split-K factor of the score sweep (second K pass)
+    bool umma;          // 128-row tiles: the full sweep runs on tcgen05 (k_umma_attn.cu)
+    bool umma_split_keys;  // tcgen05 sweep: one query tile per CTA, its two streams split the keys
+    int SU;             // tcgen05 sweep: key-range splits (S1 = SU, or 2 SU when the keys are split)
     bool mat_logits;    // hs2_step keeps the full layer's logits instead of re-reading K
     int C4;             // selected keys per sparse-attention CTA
     int S4;             // sparse-attention splits per row = ceil((k+W)/C4)
@@ -196,6 +200,8 @@ cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st);  // clears ws[
 
 cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                              cudaStream_t st);
+cudaError_t launch_umma_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
+                             cudaStream_t st);  // tensor maps with 128-key boxes
 cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st);
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);

@@ -1,0 +1,92 @@
+"""The tcgen05 full-attention sweep (128-row query tiles) against the fp64 oracle.
+
+Shapes with T * G > 64 run the full layer on the Blackwell tensor cores.  These cases cover
+both CTA modes (two query tiles sharing the K/V stream; one query tile whose two streams split
+the key range), d = 64 and 128, G = 1, 8 and 16 (128, 16 and 8 queries per tile), an odd
+number of query tiles (the last CTA's second tile is padding), key counts that are not a
+multiple of the 128-key tile, and scattered positions (rows of one tile ending in different
+key tiles, rows whose whole range lies in the first tile).  Every row's O_full and LSE_full is
+checked; the mma.sync sweep (HS2_UMMA=0) is checked on the same inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_hs2_b200 import hs2
+from long_context_sparse_hs2_b200.inputs import make_inputs
+import oracle.hs2_oracle as O
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_sparse_hs2_b200 import build
+
+    build.build()
+    hs2.lib()
+
+
+CASES = [
+    # B, Hq, Hkv, d, N, T, scattered positions
+    (1, 8, 1, 128, 5000, 16, False),    # one query tile per kv head: split-key streams, several splits
+    (2, 16, 2, 128, 3000, 40, False),   # three query tiles: pair mode, last pair half padding
+    (1, 8, 1, 64, 3000, 40, False),     # d = 64
+    (1, 4, 4, 128, 1200, 300, False),   # G = 1: 128 queries per tile
+    (1, 32, 2, 128, 2000, 20, False),   # G = 16: 8 queries per tile
+    (1, 8, 1, 128, 4100, 64, True),     # positions scattered over the whole key range
+    (2, 8, 2, 64, 700, 17, True),       # ragged: 17 queries (two tiles, second nearly empty)
+]
+
+
+def scattered_positions(B, T, N, seed):
+    rng = np.random.default_rng(seed)
+    pos = np.sort(rng.integers(0, N, size=(B, T)), axis=1).astype(np.int32)
+    pos[:, 0] = 0              # one visible key
+    pos[:, 1 % T] = min(5, N - 1)
+    pos[:, -1] = N - 1
+    return pos
+
+
+def full_rows_vs_oracle(inp, O_full, LSE_full):
+    B, Hq, T, d = inp.Qf.shape
+    Hkv = inp.K.shape[1]
+    G = Hq // Hkv
+    scale = O.softmax_scale(d)
+    Qf, K, V = O.bf16_to_f64(inp.Qf), O.bf16_to_f64(inp.K), O.bf16_to_f64(inp.V)
+    for b in range(B):
+        for h in range(Hkv):
+            hs = slice(h * G, (h + 1) * G)
+            for t in range(T):
+                p = int(inp.pos[b, t])
+                o, lse, _ = O.full_attention_row(Qf[b, hs, t], K[b, h], V[b, h], p, scale)
+                parity.assert_close_o(O_full[b, hs, t], o, f"O_full {(b, h, t)}")
+                parity.assert_close_lse(LSE_full[b, hs, t], lse, f"LSE_full {(b, h, t)}")
+
+
+@pytest.mark.parametrize("umma", ["1", "0"], ids=["tcgen05", "mma_sync"])
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+def test_full_attention_128_row_tiles(case, umma, monkeypatch):
+    monkeypatch.setenv("HS2_UMMA", umma)
+    B, Hq, Hkv, d, N, T, scattered = case
+    pos = scattered_positions(B, T, N, seed=T) if scattered else None
+    inp = make_inputs(B, Hq, Hkv, d, N, T, 16, 8, seed=N % 97, needles=4, pos=pos)
+    g = parity.gpu_inputs(inp)
+    hs2.trace_enable(True)
+    O_full, LSE_full = hs2.full_attn(g["Q_full"], g["K"], g["V"], g["pos"])
+    torch.cuda.synchronize()
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    assert ("umma_attn" in kernels) == (umma == "1"), kernels
+    full_rows_vs_oracle(inp, O_full.float().cpu().numpy(), LSE_full.cpu().numpy())
+
+
+def test_step_on_tcgen05_sweep_matches_oracle():
+    # the whole step (score re-sweep, top-k, sparse layer) on top of the tcgen05 full sweep
+    from tests.test_gpu_parity import compare_step, run_step
+
+    inp = make_inputs(1, 16, 2, 128, 2500, 24, 100, 32, seed=11, needles=6)
+    compare_step(inp, run_step(inp))
