@@ -12,18 +12,21 @@ namespace hs2 {
 
 namespace {
 
+constexpr int64_t kUmmaCtaCost = 8;  // per-CTA cost of the tcgen05 sweeps, in 128-key tiles
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Split-K factor minimising (waves x tiles per split), with a tiny penalty per split.
-int choose_splits(int64_t units, int64_t tiles, int64_t slots, int max_splits) {
+// Split-K factor minimising waves x (tiles per split + a fixed per-CTA cost in tiles: the
+// prologue, pipeline fill and partial write-out of one CTA), with a tiny penalty per split.
+int choose_splits(int64_t units, int64_t tiles, int64_t slots, int max_splits, int64_t cta_cost = 0) {
     int best = 1;
     double best_cost = 1e300;
     const int limit = static_cast<int>(std::min<int64_t>(max_splits, std::max<int64_t>(tiles, 1)));
     for (int s = 1; s <= limit; ++s) {
         const int64_t waves = (units * s + slots - 1) / slots;
-        const int64_t per = (tiles + s - 1) / s;
+        const int64_t per = (tiles + s - 1) / s + cta_cost;
         const double cost = static_cast<double>(waves * per) + 0.01 * s;
         if (cost < best_cost) {
             best_cost = cost;
@@ -79,11 +82,13 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     P.umma = P.RT == 8 && !(want_umma && want_umma[0] == '0');
     P.umma_split_keys = P.QB == 1;
     P.SU = 1;
+    P.SS = 1;
     if (P.umma) {
         const int64_t uunits = static_cast<int64_t>(x.B) * x.Hkv * (P.umma_split_keys ? P.QB : (P.QB + 1) / 2);
         const int64_t utiles = (x.N + 127) / 128;
-        P.SU = choose_splits(uunits, utiles, kSMs, 128);
+        P.SU = choose_splits(uunits, utiles, kSMs, 128, kUmmaCtaCost);
         P.S1 = P.SU * (P.umma_split_keys ? 2 : 1);
+        P.SS = choose_splits(uunits, utiles, kSMs, 256, kUmmaCtaCost);
     }
     // One decode query per batch row: the whole step can run as one kernel whose S1 x (B*Hkv)
     // CTAs are co-resident (two per SM).
@@ -241,17 +246,24 @@ TopkArgs topk_args(const Plan& p, const int32_t* pos, int32_t* idx, int32_t* cnt
 hs2_status run_select_sweep(const Plan& p, const void* Qf, const void* K, const float* LSE_full,
                             const int32_t* pos, int32_t* idx, int32_t* cnt, const Ws& w, cudaStream_t st) {
     CUtensorMap tmK;
-    if (!make_kv_map(&tmK, K, p)) return HS2_ERR_CUDA;
+    if (!make_kv_map(&tmK, K, p, p.umma ? 128 : kKeyTile)) return HS2_ERR_CUDA;
     AttnArgs a = attn_args(p, Qf, pos, w);
     a.lse = LSE_full;
     a.keys = w.at<uint32_t>(p.off_keys);
     a.kstride = p.kstride;
     a.k = p.k;
     a.S = p.S2;
-    HS2_TRY(launch_score_sweep(p, p.S2, tmK, a, st));
+    if (p.umma)
+        HS2_TRY(launch_umma_score(p, tmK, a, st));
+    else
+        HS2_TRY(launch_score_sweep(p, p.S2, tmK, a, st));
     const TopkArgs t = topk_args(p, pos, idx, cnt, w);
-    HS2_TRY(launch_topk_hist(p, t, st));
-    HS2_TRY(launch_topk_select(p, t, st));
+    if (p.rows_kv >= kRowsPerCtaTopk) {  // many rows: one CTA finishes each row
+        HS2_TRY(launch_topk_rows(p, t, st));
+    } else {
+        HS2_TRY(launch_topk_hist(p, t, st));
+        HS2_TRY(launch_topk_select(p, t, st));
+    }
     return HS2_OK;
 }
 

@@ -32,6 +32,7 @@ enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDef = 2, kMetaCand = 3, kMeta
                 kMetaSparseDone = 6, kMetaBarrier = 7 };  // kMetaDef/kMetaCand share one 8-byte word
 constexpr int kSmemCand = 4096;      // candidates the final select keeps in shared memory
 constexpr int kMaxKW = 1 << 22;      // largest supported k + W
+constexpr int kRowsPerCtaTopk = 4 * kSMs;  // from this many selection rows on, one top-k CTA per row
 
 // Everything one call needs to know about shapes, grids and workspace offsets.
 struct Plan {
@@ -46,6 +47,7 @@ struct Plan {
     bool umma;          // 128-row tiles: the full sweep runs on tcgen05 (k_umma_attn.cu)
     bool umma_split_keys;  // tcgen05 sweep: one query tile per CTA, its two streams split the keys
     int SU;             // tcgen05 sweep: key-range splits (S1 = SU, or 2 SU when the keys are split)
+    int SS;             // tcgen05 score sweep: key-range splits
     bool mat_logits;    // hs2_step keeps the full layer's logits instead of re-reading K
     int C4;             // selected keys per sparse-attention CTA
     int S4;             // sparse-attention splits per row = ceil((k+W)/C4)
@@ -202,6 +204,9 @@ cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtens
                              cudaStream_t st);
 cudaError_t launch_umma_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                              cudaStream_t st);  // tensor maps with 128-key boxes
+cudaError_t launch_umma_score(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a,
+                              cudaStream_t st);  // tensor map with 128-key boxes
+cudaError_t launch_topk_rows(const Plan& p, const TopkArgs& a, cudaStream_t st);  // one CTA per row
 cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st);
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);

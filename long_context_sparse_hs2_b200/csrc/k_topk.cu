@@ -298,6 +298,120 @@ __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
     }
 }
 
+// ====================================================================== one CTA per row (many rows)
+//
+// With thousands of selection rows (chunked prefill) one CTA finishes a whole row: it builds
+// the row's histogram in shared memory, finds the threshold bucket with a block scan, then
+// reads the row's keys again (mostly from L2) to write the keys of better buckets and collect
+// the threshold bucket's candidates in shared memory, and radix-selects the exact remainder.
+// No cross-CTA counters or global histograms.
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
+    __shared__ unsigned sh[kHistBins];
+    __shared__ unsigned long long s_cand[kSmemCand];
+    __shared__ unsigned h[256];
+    __shared__ unsigned s_small[2];
+    __shared__ unsigned s_warp[32];
+    __shared__ int s_b1, s_above, s_ndef, s_ncand, s_count;
+    static_assert(kHistBins % NT == 0 && NT % 32 == 0, "bins per thread");
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x;
+    pdl_trigger();
+    for (int i = tid; i < kHistBins; i += NT) sh[i] = 0u;
+    if (tid == 0) {
+        s_ndef = s_ncand = s_count = 0;
+        s_b1 = kHistBins;
+        s_above = -1;
+    }
+    const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
+    const int kw = a.k + a.W;
+    int32_t* idx = a.idx + row * kw;
+    int32_t* out = idx + ri.wcnt;
+    pdl_wait();  // keys from the score sweep
+    for (int i = tid; i < ri.wcnt; i += NT) idx[i] = ri.pos - ri.wcnt + 1 + i;
+    for (int i = ri.wcnt + ri.keff + tid; i < kw; i += NT) idx[i] = -1;
+    if (tid == 0) a.cnt[row] = ri.wcnt + ri.keff;
+    if (ri.keff == 0) return;
+    if (ri.keff == ri.P) {  // the whole pool is selected
+        for (int j = tid; j < ri.P; j += NT) out[j] = j;
+        return;
+    }
+    const uint32_t* keys = a.keys + row * a.kstride;
+    __syncthreads();
+    // pass 1: histogram (rows are 256-byte aligned: 16-byte loads, 4 keys each)
+    for (int base = 0; base < ri.P; base += 4 * NT) {
+        const int j = base + 4 * tid;
+        if (j < ri.P) {
+            const uint4 q = __ldcg(reinterpret_cast<const uint4*>(keys + j));
+            const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (j + e < ri.P) atomicAdd(&sh[score_bin(kk[e])], 1u);
+        }
+    }
+    __syncthreads();
+    {
+        constexpr int PER = kHistBins / NT;
+        unsigned vals[PER], sum = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            vals[i] = sh[tid * PER + i];
+            sum += vals[i];
+        }
+        const unsigned excl = block_exclusive_scan(sum, s_warp);
+        const unsigned need = static_cast<unsigned>(ri.keff);
+        if (excl < need && need <= excl + sum) {
+            unsigned cum = excl;
+            for (int i = 0; i < PER; ++i) {
+                if (cum + vals[i] >= need) {
+                    s_b1 = tid * PER + i;
+                    s_above = static_cast<int>(cum);
+                    break;
+                }
+                cum += vals[i];
+            }
+        }
+    }
+    __syncthreads();
+    const int b1 = s_b1, above = s_above;
+    if (above < 0 || above >= ri.keff) return;  // cannot happen for a consistent histogram
+    // pass 2: keys of better buckets go straight out, the threshold bucket's are candidates
+    for (int base = 0; base < ri.P; base += 4 * NT) {  // warp-uniform trip count (ballots inside)
+        const int j = base + 4 * tid;
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (j < ri.P) q = __ldcg(reinterpret_cast<const uint4*>(keys + j));
+        const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int bin = j + e < ri.P ? score_bin(kk[e]) : kHistBins;
+            const bool def = bin < b1, cnd = bin == b1;
+            const int sd = warp_append(def, &s_ndef);
+            if (def && sd < above) out[sd] = j + e;
+            const int sc = warp_append(cnd, &s_ncand);
+            if (cnd && sc < kSmemCand) s_cand[sc] = composite(kk[e], j + e);
+        }
+    }
+    __syncthreads();
+    const unsigned need = static_cast<unsigned>(ri.keff - above);
+    const int ncand = s_ncand;
+    int32_t* tail = out + above;
+    if (ncand <= kSmemCand) {
+        const SmemSource src{s_cand, ncand};
+        emit_at_least(src, radix_threshold(src, need, h, s_small), need, tail, &s_count);
+    } else {  // more ties in one bucket than shared memory holds: scan the row's keys again
+        const KeyScanSource src{keys, ri.P, b1};
+        emit_at_least(src, radix_threshold(src, need, h, s_small), need, tail, &s_count);
+    }
+}
+
+cudaError_t launch_topk_rows(const Plan& p, const TopkArgs& a, cudaStream_t st) {
+    const cudaError_t e =
+        launch_pdl(topk_rows_kernel<512>, dim3(static_cast<unsigned>(p.rows_kv)), dim3(512), 0, st, a);
+    trace_mark("topk_rows", st);
+    return e;
+}
+
 cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st) {
     dim3 grid((p.N + kTopkChunk - 1) / kTopkChunk, static_cast<unsigned>(p.rows_kv));
     const cudaError_t e = launch_pdl(topk_hist_kernel, grid, dim3(256), 0, st, a);

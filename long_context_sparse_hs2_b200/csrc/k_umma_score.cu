@@ -1,0 +1,287 @@
+// Selection-score sweep on the Blackwell tensor cores (tcgen05 / TMEM) for 128-row query tiles.
+//
+// The second K pass computes, for every query and pool key j <= pos - W, the GQA-max
+// log-softmax score s_j = max over the G heads g of (logit_gj - LSE_g) in base-2 units and
+// stores it as an order-preserving uint32 key for the top-k.  Here the product is taken
+// transposed, S^T = K Q^T: the M dimension is 128 keys (one TMEM lane, one epilogue thread per
+// key) and the N dimension the query-head rows of one or two query tiles (row = query * G +
+// head, N = 128 or 256).  A thread then holds all G heads of every query for its key in its
+// own registers, so the max over heads needs no shuffles, and the 32 threads of a warp write
+// 32 consecutive keys of one query (128-byte stores).
+//
+// With x = q . k (the raw dot product), logit - LSE in base 2 is c * (x - u) for
+// c = log2(e) / sqrt(d) and u = LSE * sqrt(d) (natural-log LSE), so the epilogue subtracts a
+// per-row constant, takes the max over heads, and scales once per (query, key).
+//
+// Roles (320 threads): warps 0-3 and 4-7 are two epilogue warpgroups working on alternate key
+// tiles, each with its own TMEM accumulator (256 columns); warp 8 streams K tiles of 128 keys
+// (4-stage TMA ring); warp 9 allocates TMEM and one of its lanes issues the MMAs.  Every wait
+// is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains and exits.
+#include "attn_sweep.cuh"
+#include "umma.cuh"
+
+namespace hs2 {
+
+namespace {
+
+constexpr int kSTile = 128;      // keys per K tile (= TMEM lanes = M)
+constexpr int kURowsPerTile = 128;  // query-head rows per query tile
+constexpr int kSStages = 4;
+constexpr int kSThreads = 320;
+constexpr int kSMaxCols = 256;   // query-head rows per CTA (two query tiles)
+
+template <int D>
+struct SSmem {
+    static constexpr int kQBytes = kSMaxCols * D * 2;    // both query tiles, [D/64][256 rows][128 B]
+    static constexpr int kQHalf = kSMaxCols * 128;
+    static constexpr int kTileBytes = kSTile * D * 2;
+    static constexpr int kBlock = kSTile * 128;          // one 64-column block of a K tile
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQBytes;
+    static constexpr int kBarOff = kKOff + kSStages * kTileBytes;
+    static constexpr int kNumBars = 2 * kSStages + 5;    // kfull, kempty, sfull[2], tfree[2], done
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kUOff = kMiscOff + 16;          // u per column (float)
+    static constexpr int kPlOff = kUOff + kSMaxCols * 4; // last pool key per query (-1: none)
+    static constexpr int kRowOff = kPlOff + kSMaxCols * 4;  // selection row per query
+    static constexpr int kBytes = kRowOff + kSMaxCols * 4 + 1024;
+};
+
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+}  // namespace
+
+template <int D, int G>
+__global__ void __launch_bounds__(kSThreads, 1)
+    umma_score_kernel(const __grid_constant__ CUtensorMap tmK, const AttnArgs a, const int split_keys) {
+    using L = SSmem<D>;
+    constexpr int TQ = kURowsPerTile / G;  // queries per query tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* kfull = bars;
+    uint64_t* kempty = bars + kSStages;
+    uint64_t* sfull = bars + 2 * kSStages;
+    uint64_t* tfree = sfull + 2;
+    uint64_t* done = sfull + 4;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+    float* s_u = reinterpret_cast<float*>(smem + L::kUOff);
+    int* s_pl = reinterpret_cast<int*>(smem + L::kPlOff);
+    int* s_row = reinterpret_cast<int*>(smem + L::kRowOff);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_trigger();
+    const int split = blockIdx.x, unit = blockIdx.y;
+    const int QP = split_keys ? a.QB : (a.QB + 1) / 2;
+    const int bh = unit / QP, pr = unit % QP;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const int nq = split_keys ? 1 : 2;
+    const int ncols = nq * kURowsPerTile;
+
+    // ---- prologue: per-query pool ends and rows, query tiles (swizzled), barriers
+    for (int qa = tid; qa < nq * TQ; qa += kSThreads) {
+        const int s = qa / TQ, tq = qa % TQ;
+        const int qb = split_keys ? pr : 2 * pr + s;
+        const int t = qb * TQ + tq;
+        int pl = -1;
+        if (qb < a.QB && t < a.T) {
+            const int p = clamp_pos(a.pos[b * a.T + t], a.N, nullptr);
+            const int P = max(0, p - a.W + 1);
+            const int keff = min(a.k, P);
+            if (keff > 0 && keff < P) pl = p - a.W;  // only these rows need ranked keys
+        }
+        s_pl[qa] = pl;
+        s_row[qa] = bh * a.T + t;
+    }
+    constexpr int CH = D / 8;
+    for (int i = tid; i < nq * kURowsPerTile * CH; i += kSThreads) {
+        const int R = i / CH, c = i % CH;  // R = s * 128 + r
+        const int s = R / kURowsPerTile, r = R % kURowsPerTile;
+        const int qb = split_keys ? pr : 2 * pr + s;
+        const int tq = r / G, t = qb * TQ + tq;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (qb < a.QB && t < a.T) {
+            const int64_t grow = static_cast<int64_t>((b * a.Hq + h * G + r % G)) * a.T + t;
+            v = *reinterpret_cast<const uint4*>(a.Q + grow * D + c * 8);
+        }
+        *reinterpret_cast<uint4*>(smem + L::kQOff + (c >> 3) * L::kQHalf + R * 128 + (((c & 7) ^ (R & 7)) << 4)) = v;
+    }
+    fence_async_smem();
+    if (tid == 0) {
+        for (int i = 0; i < L::kNumBars; ++i) {
+            const bool is_tfree = i >= 2 * kSStages + 2 && i < 2 * kSStages + 4;
+            mbar_init(&bars[i], is_tfree ? kSTile : 1);  // tfree: one arrival per epilogue thread
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    pdl_wait();  // LSE_full comes from the previous kernel; TMEM only after it has completed
+    __syncthreads();  // s_pl complete
+    const float sqrt_d = sqrtf(static_cast<float>(D));
+    for (int col = tid; col < kSMaxCols; col += kSThreads) {
+        float u = INFINITY;  // padding or unranked rows: every score -inf, never written
+        if (col < ncols) {
+            const int s = col / kURowsPerTile, r = col % kURowsPerTile;
+            const int qa = s * TQ + r / G;
+            if (s_pl[qa] >= 0) {
+                const int qb = split_keys ? pr : 2 * pr + s;
+                const int t = qb * TQ + r / G;
+                u = a.lse[static_cast<int64_t>(b * a.Hq + h * G + r % G) * a.T + t] * sqrt_d;
+            }
+        }
+        s_u[col] = u;
+    }
+    if (warp == 9) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *s_tmem;
+
+    int jmax = -1;
+    for (int qa = 0; qa < nq * TQ; ++qa) jmax = max(jmax, s_pl[qa]);
+    const int ntiles = jmax >= 0 ? (jmax + kSTile) / kSTile : 0;
+    const int t_begin = static_cast<int>((static_cast<int64_t>(split) * ntiles) / a.S);
+    const int t_end = static_cast<int>((static_cast<int64_t>(split + 1) * ntiles) / a.S);
+    const int nt = t_end - t_begin;
+
+    bool nonfinite = false;
+    if (warp == 8) {
+        // ------------------------------------------------------------ TMA producer (K only)
+        if (lane == 0) {
+            const uint64_t pol = a.stream_kv ? l2_evict_first() : l2_evict_normal();
+            prefetch_tensormap(&tmK);
+            int issued = 0;
+            for (int q = 0; q < nt; ++q) {
+                const int st = q % kSStages;
+                if (q >= kSStages && !mbar_wait(&kempty[st], ((q / kSStages) - 1) & 1, a.status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                mbar_arrive_expect_tx(&kfull[st], L::kTileBytes);
+#pragma unroll
+                for (int hb = 0; hb < D / 64; ++hb)
+                    tma_load_3d(smem + L::kKOff + st * L::kTileBytes + hb * L::kBlock, &tmK, &kfull[st], hb * 64,
+                                (t_begin + q) * kSTile, bh, pol);
+                ++issued;
+            }
+            for (int st = 0; st < kSStages && st < issued; ++st) {
+                const int last = st + ((issued - 1 - st) / kSStages) * kSStages;
+                mbar_wait(&kfull[st], (last / kSStages) & 1, a.status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kSTile, ncols, false);
+            const uint32_t qb0 = smem_u32(smem + L::kQOff);
+            const uint32_t kb0 = smem_u32(smem + L::kKOff);
+            bool ok = true;
+            for (int i = 0; ok && i < nt; ++i) {
+                const int st = i % kSStages, buf = i & 1;
+                ok = !*abort_flag && mbar_wait(&kfull[st], (i / kSStages) & 1, a.status);
+                if (ok && i >= 2) ok = mbar_wait(&tfree[buf], ((i >> 1) - 1) & 1, a.status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t kb = kb0 + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * L::kBlock + (kk & 3) * 32;
+                    const uint32_t qoff = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
+                    umma_ss(tm + 256 * buf, sw128_desc(kb + koff, 16, 1024), sw128_desc(qb0 + qoff, 16, 1024), idesc,
+                            kk > 0);
+                }
+                umma_commit(&kempty[st]);
+                umma_commit(&sfull[buf]);
+            }
+            if (!ok) *abort_flag = 1;
+            umma_commit(done);
+            mbar_wait(done, 0, a.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (thread = key)
+        const int w = warp >> 2, quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t tbase = tm + (static_cast<uint32_t>(quarter * 32) << 16) + 256 * w;
+        const float c2 = a.scale_log2;
+        for (int i = w; i < nt; i += 2) {
+            const bool got = mbar_wait(&sfull[w], (i >> 1) & 1, a.status);
+            if (!got) *abort_flag = 1;
+            if (!__all_sync(0xffffffffu, got && !*abort_flag)) break;
+            tc_fence_after();
+            const int j = (t_begin + i) * kSTile + r;
+            for (int c0 = 0; c0 < ncols; c0 += 64) {
+                uint32_t x[2][32];
+                tmem_ld32(tbase + c0, x[0]);
+                tmem_ld32(tbase + c0 + 32, x[1]);
+                tmem_wait_ld();
+                tie_regs(x[0]);
+                tie_regs(x[1]);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int qq = 0; qq < 32 / G; ++qq) {
+                        const int col = c0 + 32 * hh + qq * G;
+                        float m = -INFINITY;
+#pragma unroll
+                        for (int g = 0; g < G; ++g) m = max_nan(m, __uint_as_float(x[hh][qq * G + g]) - s_u[col + g]);
+                        const int qa = col / G;
+                        if (j <= s_pl[qa]) {
+                            const float sv = m * c2;
+                            nonfinite |= (sv != sv);
+                            a.keys[static_cast<int64_t>(s_row[qa]) * a.kstride + j] = score_key(sv);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tfree[w]);
+        }
+    }
+
+    tc_fence_before();
+    if (__syncthreads_or(nonfinite) && tid == 0) set_status(a.status, HS2_DEV_NONFINITE);
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+// ====================================================================== launcher
+
+template <int D, int G>
+cudaError_t umma_score_variant(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st) {
+    using L = SSmem<D>;
+    auto kern = umma_score_kernel<D, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+    const int split_keys = p.umma_split_keys ? 1 : 0;
+    const int QP = split_keys ? p.QB : (p.QB + 1) / 2;
+    dim3 grid(p.SS, p.B * p.Hkv * QP);
+    AttnArgs x = a;
+    x.S = p.SS;
+    e = launch_pdl(kern, grid, dim3(kSThreads), L::kBytes, st, tmK, x, split_keys);
+    trace_mark("umma_score", st);
+    return e;
+}
+
+cudaError_t launch_umma_score(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a, cudaStream_t st) {
+#define HS2_US(D_, G_) \
+    if (p.d == D_ && p.G == G_) return umma_score_variant<D_, G_>(p, tmK, a, st);
+    HS2_US(128, 1) HS2_US(128, 2) HS2_US(128, 4) HS2_US(128, 8) HS2_US(128, 16)
+    HS2_US(64, 1) HS2_US(64, 2) HS2_US(64, 4) HS2_US(64, 8) HS2_US(64, 16)
+#undef HS2_US
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace hs2

@@ -84,9 +84,53 @@ def test_full_attention_128_row_tiles(case, umma, monkeypatch):
     full_rows_vs_oracle(inp, O_full.float().cpu().numpy(), LSE_full.cpu().numpy())
 
 
-def test_step_on_tcgen05_sweep_matches_oracle():
-    # the whole step (score re-sweep, top-k, sparse layer) on top of the tcgen05 full sweep
+STEP_CASES = [
+    # B, Hq, Hkv, d, N, T, k, W, scattered positions
+    (1, 16, 2, 128, 2500, 24, 100, 32, False),   # G = 8, pair mode
+    (2, 16, 2, 128, 3000, 16, 64, 16, False),    # split mode, two batch rows
+    (1, 4, 4, 128, 1200, 300, 50, 16, False),    # G = 1
+    (1, 32, 2, 64, 2000, 20, 64, 8, False),      # G = 16, d = 64
+    (1, 8, 1, 128, 4100, 64, 300, 64, True),     # scattered: unranked rows (pos < W, k >= pool)
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=[str(c) for c in STEP_CASES])
+def test_step_on_tcgen05_sweeps_matches_oracle(case):
+    # the whole step on the tcgen05 full and score sweeps, then top-k and the sparse layer
     from tests.test_gpu_parity import compare_step, run_step
 
-    inp = make_inputs(1, 16, 2, 128, 2500, 24, 100, 32, seed=11, needles=6)
-    compare_step(inp, run_step(inp))
+    B, Hq, Hkv, d, N, T, k, W, scattered = case
+    pos = scattered_positions(B, T, N, seed=T + 1) if scattered else None
+    inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=T + N % 31, needles=6, pos=pos)
+    hs2.trace_enable(True)
+    res = run_step(inp)
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    assert "umma_attn" in kernels and "umma_score" in kernels, kernels
+    compare_step(inp, res)
+
+
+def test_many_rows_one_cta_per_row_topk():
+    # >= 592 selection rows: the top-k runs one CTA per row (histogram, threshold, emit, radix)
+    from tests.test_gpu_parity import compare_step, run_step
+
+    inp = make_inputs(1, 32, 4, 128, 3000, 160, 64, 16, seed=21, needles=8)
+    hs2.trace_enable(True)
+    res = run_step(inp)
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    assert "topk_rows" in kernels, kernels
+    compare_step(inp, res)
+
+
+def test_many_rows_all_scores_equal():
+    # Q = 0: every pool key ties, far more candidates than shared memory holds (key re-scan
+    # path); the k lowest indices must win in every row
+    from tests.test_gpu_parity import compare_step, run_step
+
+    inp = make_inputs(1, 16, 2, 128, 6000, 320, 100, 10, seed=22)
+    inp.Qf = np.zeros_like(inp.Qf)
+    res = run_step(inp)
+    ref = compare_step(inp, res)
+    for (b, h, t), r in ref.items():
+        np.testing.assert_array_equal(np.sort(res["idx"][b, h, t][:res["cnt"][b, h, t]]), r.selected)
