@@ -16,11 +16,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kKeyTile = 64;                      // keys per K/V shared-memory tile
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bound on any single pipeline wait (2 s)
 constexpr int kSMs = 148;            // B200 streaming multiprocessors
-constexpr int kHistBins = 2048;      // top-k histogram: 1/32 of a base-2 score unit per bin
-constexpr float kBinsPerUnit = 32.f;
+constexpr int kHistBins = 2048;      // top-k histogram buckets (see score_bin)
 constexpr int kTopkChunk = 4096;     // pool keys per CTA in the histogram / emit passes
 constexpr int kMetaInts = 8;
-constexpr int kSweepMaxTiles = 65535 / 64;  // tiles per score-sweep CTA (16-bit histogram counters)         // per-row top-k bookkeeping ints (see TopkMeta)
 
 // Per-row bookkeeping in the workspace (ints; zeroed before each use, see Plan::off_meta).
 //   kMetaBin / kMetaAbove: threshold bucket of the k-th best key and the count above it

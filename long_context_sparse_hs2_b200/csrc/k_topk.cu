@@ -376,20 +376,51 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
     __syncthreads();
     const int b1 = s_b1, above = s_above;
     if (above < 0 || above >= ri.keff) return;  // cannot happen for a consistent histogram
-    // pass 2: keys of better buckets go straight out, the threshold bucket's are candidates
-    for (int base = 0; base < ri.P; base += 4 * NT) {  // warp-uniform trip count (ballots inside)
+    // pass 2: keys of better buckets go straight out, the threshold bucket's are candidates.
+    // Each thread has 4 keys; a warp with any hit scans its per-lane counts (packed: defs in the
+    // low, candidates in the high half-word) and reserves its slots with one shared-memory
+    // atomic per list.
+    const int lane = tid & 31;
+    for (int base = 0; base < ri.P; base += 4 * NT) {  // warp-uniform trip count (shuffles inside)
         const int j = base + 4 * tid;
         uint4 q = make_uint4(0u, 0u, 0u, 0u);
         if (j < ri.P) q = __ldcg(reinterpret_cast<const uint4*>(keys + j));
         const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+        unsigned dmask = 0u, cmask = 0u;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int bin = j + e < ri.P ? score_bin(kk[e]) : kHistBins;
-            const bool def = bin < b1, cnd = bin == b1;
-            const int sd = warp_append(def, &s_ndef);
-            if (def && sd < above) out[sd] = j + e;
-            const int sc = warp_append(cnd, &s_ncand);
-            if (cnd && sc < kSmemCand) s_cand[sc] = composite(kk[e], j + e);
+            dmask |= static_cast<unsigned>(bin < b1) << e;
+            cmask |= static_cast<unsigned>(bin == b1) << e;
+        }
+        if (!__any_sync(0xffffffffu, (dmask | cmask) != 0u)) continue;
+        const unsigned mine = __popc(dmask) | (__popc(cmask) << 16);  // <= 128 per warp: no carry
+        unsigned incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int bdef = 0, bcnd = 0;
+        if (lane == 31) {
+            if (incl & 0xFFFFu) bdef = atomicAdd(&s_ndef, static_cast<int>(incl & 0xFFFFu));
+            if (incl >> 16) bcnd = atomicAdd(&s_ncand, static_cast<int>(incl >> 16));
+        }
+        bdef = __shfl_sync(0xffffffffu, bdef, 31);
+        bcnd = __shfl_sync(0xffffffffu, bcnd, 31);
+        const unsigned excl = incl - mine;
+        int od = bdef + static_cast<int>(excl & 0xFFFFu);
+        int oc = bcnd + static_cast<int>(excl >> 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (dmask >> e & 1u) {
+                if (od < above) out[od] = j + e;
+                ++od;
+            }
+            if (cmask >> e & 1u) {
+                if (oc < kSmemCand) s_cand[oc] = composite(kk[e], j + e);
+                ++oc;
+            }
         }
     }
     __syncthreads();

@@ -10,13 +10,17 @@
 // 32 consecutive keys of one query (128-byte stores).
 //
 // With x = q . k (the raw dot product), logit - LSE in base 2 is c * (x - u) for
-// c = log2(e) / sqrt(d) and u = LSE * sqrt(d) (natural-log LSE), so the epilogue subtracts a
-// per-row constant, takes the max over heads, and scales once per (query, key).
+// c = log2(e) / sqrt(d) and u = LSE * sqrt(d) (natural-log LSE).  The subtraction is folded
+// into the MMA: one extra K step multiplies a constant key block (1, 1, 1, 0, ...) with a
+// per-row block (-u split into three bf16 parts whose sum is u to about 24 bits), so TMEM
+// already holds x - u and the epilogue is a max over heads and one scale per (query, key).
 //
-// Roles (320 threads): warps 0-3 and 4-7 are two epilogue warpgroups working on alternate key
-// tiles, each with its own TMEM accumulator (256 columns); warp 8 streams K tiles of 128 keys
-// (4-stage TMA ring); warp 9 allocates TMEM and one of its lanes issues the MMAs.  Every wait
-// is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains and exits.
+// Roles (320 threads): warps 0-3 and 4-7 are two epilogue warpgroups that split the columns
+// of every tile between them (one query tile each, or half of one); two TMEM accumulators
+// (256 columns each) let the MMA of tile i + 1 run during the epilogue of tile i; warp 8
+// streams K tiles of 128 keys (3-stage TMA ring); warp 9 allocates TMEM and one of its lanes
+// issues the MMAs.  Every wait is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains
+// and exits.
 #include "attn_sweep.cuh"
 #include "umma.cuh"
 
@@ -26,7 +30,7 @@ namespace {
 
 constexpr int kSTile = 128;      // keys per K tile (= TMEM lanes = M)
 constexpr int kURowsPerTile = 128;  // query-head rows per query tile
-constexpr int kSStages = 4;
+constexpr int kSStages = 3;
 constexpr int kSThreads = 320;
 constexpr int kSMaxCols = 256;   // query-head rows per CTA (two query tiles)
 
@@ -37,14 +41,14 @@ struct SSmem {
     static constexpr int kTileBytes = kSTile * D * 2;
     static constexpr int kBlock = kSTile * 128;          // one 64-column block of a K tile
     static constexpr int kQOff = 0;
-    static constexpr int kKOff = kQBytes;
+    static constexpr int kQcOff = kQBytes;               // -u parts per row: [256 rows][128 B] (16 B used)
+    static constexpr int kKcOff = kQcOff + kSMaxCols * 128;  // ones per key: [128 keys][128 B]
+    static constexpr int kKOff = kKcOff + kSTile * 128;
     static constexpr int kBarOff = kKOff + kSStages * kTileBytes;
     static constexpr int kNumBars = 2 * kSStages + 5;    // kfull, kempty, sfull[2], tfree[2], done
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kUOff = kMiscOff + 16;          // u per column (float)
-    static constexpr int kPlOff = kUOff + kSMaxCols * 4; // last pool key per query (-1: none)
-    static constexpr int kRowOff = kPlOff + kSMaxCols * 4;  // selection row per query
-    static constexpr int kBytes = kRowOff + kSMaxCols * 4 + 1024;
+    static constexpr int kPlOff = kMiscOff + 16;         // last pool key per query (-1: not ranked)
+    static constexpr int kBytes = kPlOff + kSMaxCols * 4 + 1024;
 };
 
 __device__ __forceinline__ float max_nan(float a, float b) {
@@ -52,6 +56,13 @@ __device__ __forceinline__ float max_nan(float a, float b) {
     asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
     return r;
 }
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(r) : "f"(x));
+    return static_cast<uint16_t>(r & 0xFFFFu);
+}
+__device__ __forceinline__ float bf16_value(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
 }  // namespace
 
@@ -70,9 +81,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     uint64_t* done = sfull + 4;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-    float* s_u = reinterpret_cast<float*>(smem + L::kUOff);
     int* s_pl = reinterpret_cast<int*>(smem + L::kPlOff);
-    int* s_row = reinterpret_cast<int*>(smem + L::kRowOff);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_trigger();
@@ -83,7 +92,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     const int nq = split_keys ? 1 : 2;
     const int ncols = nq * kURowsPerTile;
 
-    // ---- prologue: per-query pool ends and rows, query tiles (swizzled), barriers
+    // ---- prologue: per-query pool ends, query tiles and the constant key block (swizzled)
     for (int qa = tid; qa < nq * TQ; qa += kSThreads) {
         const int s = qa / TQ, tq = qa % TQ;
         const int qb = split_keys ? pr : 2 * pr + s;
@@ -96,7 +105,6 @@ __global__ void __launch_bounds__(kSThreads, 1)
             if (keff > 0 && keff < P) pl = p - a.W;  // only these rows need ranked keys
         }
         s_pl[qa] = pl;
-        s_row[qa] = bh * a.T + t;
     }
     constexpr int CH = D / 8;
     for (int i = tid; i < nq * kURowsPerTile * CH; i += kSThreads) {
@@ -111,11 +119,15 @@ __global__ void __launch_bounds__(kSThreads, 1)
         }
         *reinterpret_cast<uint4*>(smem + L::kQOff + (c >> 3) * L::kQHalf + R * 128 + (((c & 7) ^ (R & 7)) << 4)) = v;
     }
-    fence_async_smem();
+    for (int i = tid; i < kSTile * 8; i += kSThreads) {  // key block: elements 0..2 of every row are 1
+        const int r = i >> 3, c = i & 7;
+        const uint4 v = c == 0 ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + L::kKcOff + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
     if (tid == 0) {
         for (int i = 0; i < L::kNumBars; ++i) {
             const bool is_tfree = i >= 2 * kSStages + 2 && i < 2 * kSStages + 4;
-            mbar_init(&bars[i], is_tfree ? kSTile : 1);  // tfree: one arrival per epilogue thread
+            mbar_init(&bars[i], is_tfree ? 2 * kSTile : 1);  // tfree: one arrival per epilogue thread
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -123,19 +135,26 @@ __global__ void __launch_bounds__(kSThreads, 1)
     pdl_wait();  // LSE_full comes from the previous kernel; TMEM only after it has completed
     __syncthreads();  // s_pl complete
     const float sqrt_d = sqrtf(static_cast<float>(D));
-    for (int col = tid; col < kSMaxCols; col += kSThreads) {
-        float u = INFINITY;  // padding or unranked rows: every score -inf, never written
-        if (col < ncols) {
-            const int s = col / kURowsPerTile, r = col % kURowsPerTile;
+    for (int i = tid; i < kSMaxCols * 8; i += kSThreads) {  // row block: -u as hi + mid + lo
+        const int R = i >> 3, c = i & 7;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (c == 0 && R < ncols) {
+            const int s = R / kURowsPerTile, r = R % kURowsPerTile;
             const int qa = s * TQ + r / G;
-            if (s_pl[qa] >= 0) {
+            if (s_pl[qa] >= 0) {  // unranked and padding rows keep u = 0: never written
                 const int qb = split_keys ? pr : 2 * pr + s;
                 const int t = qb * TQ + r / G;
-                u = a.lse[static_cast<int64_t>(b * a.Hq + h * G + r % G) * a.T + t] * sqrt_d;
+                const float nu = -a.lse[static_cast<int64_t>(b * a.Hq + h * G + r % G) * a.T + t] * sqrt_d;
+                const uint16_t hi = bf16_bits_rn(nu);
+                const float r1 = nu - bf16_value(hi);
+                const uint16_t mid = bf16_bits_rn(r1);
+                const uint16_t lo = bf16_bits_rn(r1 - bf16_value(mid));
+                v = make_uint4(static_cast<uint32_t>(hi) | (static_cast<uint32_t>(mid) << 16), lo, 0u, 0u);
             }
         }
-        s_u[col] = u;
+        *reinterpret_cast<uint4*>(smem + L::kQcOff + R * 128 + ((c ^ (R & 7)) << 4)) = v;
     }
+    fence_async_smem();
     if (warp == 9) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
@@ -185,6 +204,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
             const uint32_t idesc = idesc_bf16(kSTile, ncols, false);
             const uint32_t qb0 = smem_u32(smem + L::kQOff);
             const uint32_t kb0 = smem_u32(smem + L::kKOff);
+            const uint64_t kc_desc = sw128_desc(smem_u32(smem + L::kKcOff), 16, 1024);
+            const uint64_t qc_desc = sw128_desc(smem_u32(smem + L::kQcOff), 16, 1024);
             bool ok = true;
             for (int i = 0; ok && i < nt; ++i) {
                 const int st = i % kSStages, buf = i & 1;
@@ -200,6 +221,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
                     umma_ss(tm + 256 * buf, sw128_desc(kb + koff, 16, 1024), sw128_desc(qb0 + qoff, 16, 1024), idesc,
                             kk > 0);
                 }
+                umma_ss(tm + 256 * buf, kc_desc, qc_desc, idesc, 1u);  // - u
                 umma_commit(&kempty[st]);
                 umma_commit(&sfull[buf]);
             }
@@ -212,18 +234,31 @@ __global__ void __launch_bounds__(kSThreads, 1)
         // ------------------------------------------------------------ epilogue (thread = key)
         const int w = warp >> 2, quarter = warp & 3;
         const int r = quarter * 32 + lane;
-        const uint32_t tbase = tm + (static_cast<uint32_t>(quarter * 32) << 16) + 256 * w;
+        const int wcols = ncols / 2;           // columns of this warpgroup: one query tile, or half of one
+        const int col0 = w * wcols;
+        const int s = col0 / kURowsPerTile;    // query tile of these columns
+        const int qa0 = col0 / G, nqw = wcols / G;
+        const int qb = split_keys ? pr : 2 * pr + s;
+        // selection row of query qa0 + i is row0 + i (valid queries only; the others are never written)
+        const int64_t row0 = static_cast<int64_t>(bh) * a.T + qb * TQ + (qa0 - s * TQ);
+        int plmin = INT_MAX;
+        for (int i = 0; i < nqw; ++i) plmin = min(plmin, s_pl[qa0 + i]);  // -1 if any is not ranked
+        const uint32_t tbase = tm + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
         const float c2 = a.scale_log2;
-        for (int i = w; i < nt; i += 2) {
-            const bool got = mbar_wait(&sfull[w], (i >> 1) & 1, a.status);
+        for (int i = 0; i < nt; ++i) {
+            const int buf = i & 1;
+            const bool got = mbar_wait(&sfull[buf], (i >> 1) & 1, a.status);
             if (!got) *abort_flag = 1;
             if (!__all_sync(0xffffffffu, got && !*abort_flag)) break;
             tc_fence_after();
-            const int j = (t_begin + i) * kSTile + r;
-            for (int c0 = 0; c0 < ncols; c0 += 64) {
+            const int jt = (t_begin + i) * kSTile;
+            const int j = jt + r;
+            const bool fast = jt + kSTile - 1 <= plmin;  // every query of these columns takes every key
+            uint32_t* kp = a.keys + row0 * a.kstride + j;
+            for (int c0 = 0; c0 < wcols; c0 += 64) {
                 uint32_t x[2][32];
-                tmem_ld32(tbase + c0, x[0]);
-                tmem_ld32(tbase + c0 + 32, x[1]);
+                tmem_ld32(tbase + 256 * buf + c0, x[0]);
+                tmem_ld32(tbase + 256 * buf + c0 + 32, x[1]);
                 tmem_wait_ld();
                 tie_regs(x[0]);
                 tie_regs(x[1]);
@@ -231,21 +266,20 @@ __global__ void __launch_bounds__(kSThreads, 1)
                 for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
                     for (int qq = 0; qq < 32 / G; ++qq) {
-                        const int col = c0 + 32 * hh + qq * G;
-                        float m = -INFINITY;
+                        float m = __uint_as_float(x[hh][qq * G]);
 #pragma unroll
-                        for (int g = 0; g < G; ++g) m = max_nan(m, __uint_as_float(x[hh][qq * G + g]) - s_u[col + g]);
-                        const int qa = col / G;
-                        if (j <= s_pl[qa]) {
+                        for (int g = 1; g < G; ++g) m = max_nan(m, __uint_as_float(x[hh][qq * G + g]));
+                        const int qi = (c0 + 32 * hh) / G + qq;  // query index within these columns
+                        if (fast || j <= s_pl[qa0 + qi]) {
                             const float sv = m * c2;
                             nonfinite |= (sv != sv);
-                            a.keys[static_cast<int64_t>(s_row[qa]) * a.kstride + j] = score_key(sv);
+                            kp[static_cast<int64_t>(qi) * a.kstride] = score_key(sv);
                         }
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(&tfree[w]);
+            mbar_arrive(&tfree[buf]);
         }
     }
 

@@ -1,11 +1,15 @@
 // Pieces of the exact token-level top-k shared by the scoring and selection kernels.
 //
 // Keys: the fp32 score s (base-2 units) maps to an order-preserving uint32 (score_key).
-// Buckets: score_bin is a monotone, non-increasing function of the score with 1/32 of a
-// base-2 unit per bin (bin 0 = best, NaN last), so every key in a better bucket than the
-// bucket holding the k-th best key is selected outright.  Composite: (key << 32) |
-// (2^32 - 1 - j) is distinct per key and orders by (score desc, index asc) -- exactly the
-// selection rule with ties to the lower index.
+// Buckets: score_bin is a monotone, non-increasing function of the score, read straight from
+// the key's bits: a selection score is a log-probability (<= 0), and for s < 0 the key is
+// 0x7FFFFFFF - bits(|s|), so bits(|s|) >> 15 (exponent and 8 mantissa bits) is a logarithmic
+// bucket of |s| with 256 buckets per octave.  Buckets 0 .. 2047 cover |s| in [1/4, 64) (1/32
+// of a unit per bucket around |s| = 8); |s| < 1/4 and s >= 0 share bucket 0, |s| >= 64 and
+// NaN (key 0) the last one.  Every key in a better bucket than the bucket holding the k-th
+// best key is selected outright.  Composite: (key << 32) | (2^32 - 1 - j) is distinct per
+// key and orders by (score desc, index asc) -- exactly the selection rule with ties to the
+// lower index.
 #pragma once
 
 #include "hs2_device.cuh"
@@ -13,11 +17,9 @@
 namespace hs2 {
 
 __device__ __forceinline__ int score_bin(uint32_t key) {
-    if (key == 0u) return kHistBins - 1;  // NaN ranks last
-    const float x = -key_score(key) * kBinsPerUnit;
-    if (!(x > 0.f)) return 0;
-    if (x >= static_cast<float>(kHistBins - 1)) return kHistBins - 1;
-    return static_cast<int>(x);
+    constexpr int kFirst = (125 << 8);  // bits(0.25) >> 15
+    const int v = (static_cast<int>(0x7FFFFFFFu - key) >> 15) - kFirst;  // negative for s >= 0
+    return min(max(v, 0), kHistBins - 1);
 }
 
 __device__ __forceinline__ unsigned long long composite(uint32_t key, int j) {
