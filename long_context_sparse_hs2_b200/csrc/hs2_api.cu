@@ -85,10 +85,10 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     P.SS = 1;
     if (P.umma) {
         const int64_t uunits = static_cast<int64_t>(x.B) * x.Hkv * (P.umma_split_keys ? P.QB : (P.QB + 1) / 2);
-        const int64_t utiles = (x.N + 127) / 128;
-        P.SU = choose_splits(uunits, utiles, kSMs, 128, kUmmaCtaCost);
+        const int64_t tiles128 = (x.N + 127) / 128;
+        P.SU = choose_splits(uunits, tiles128, kSMs, 128, kUmmaCtaCost);
         P.S1 = P.SU * (P.umma_split_keys ? 2 : 1);
-        P.SS = choose_splits(uunits, utiles, kSMs, 256, kUmmaCtaCost);
+        P.SS = choose_splits(uunits, tiles128, kSMs, 256, kUmmaCtaCost);
     }
     // One decode query per batch row: the whole step can run as one kernel whose S1 x (B*Hkv)
     // CTAs are co-resident (two per SM).
@@ -103,7 +103,9 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     const int64_t kw = static_cast<int64_t>(x.k) + x.W;
     const int64_t s4_target = std::max<int64_t>(1, kSMs / rows_kv);
     const int64_t c4 = ((std::max<int64_t>(1, (kw + s4_target - 1) / s4_target) + 63) / 64) * 64;
-    P.C4 = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(64, c4)));
+    // with many rows every CTA takes a whole row (up to kSparseMaxC4 keys): no split partials
+    const int64_t c4_cap = rows_kv >= 2 * kSMs ? kSparseMaxC4 : 1024;
+    P.C4 = static_cast<int>(std::min<int64_t>(c4_cap, std::max<int64_t>(64, c4)));
     P.S4 = static_cast<int>(std::max<int64_t>(1, (kw + P.C4 - 1) / P.C4));
     // combine scratch: the sparse combine keeps G * S4 weights in the gather ring, the score
     // kernel's combine CTA G * S1 weights in its histogram scratch

@@ -30,6 +30,7 @@ enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDef = 2, kMetaCand = 3, kMeta
                 kMetaSparseDone = 6, kMetaBarrier = 7 };  // kMetaDef/kMetaCand share one 8-byte word
 constexpr int kSmemCand = 4096;      // candidates the final select keeps in shared memory
 constexpr int kMaxKW = 1 << 22;      // largest supported k + W
+constexpr int kSparseMaxC4 = 4096;         // most selected keys one sparse-attention CTA takes
 constexpr int kRowsPerCtaTopk = 4 * kSMs;  // from this many selection rows on, one top-k CTA per row
 
 // Everything one call needs to know about shapes, grids and workspace offsets.

@@ -27,7 +27,7 @@ constexpr int kSparseWarps = 8;
 constexpr int kSparseThreads = kSparseWarps * 32;
 constexpr int kSparseTile = 2 * kKeyTile;  // keys per pipeline step: two 64-key sub-tiles
 
-constexpr int kSparseStages = 2;
+constexpr int kSparseStages = 3;
 
 template <int D>
 struct SparseSmem {
@@ -39,11 +39,15 @@ struct SparseSmem {
     static constexpr int bytes(int C4) { return kIdxOff + (C4 + kSparseTile) * 4 + 16 + 1024; }
 };
 
+// Wait until at most `pending` of this thread's cp.async groups are still in flight.
 __device__ __forceinline__ void cp_async_wait_upto(int pending) {
+    static_assert(kSparseStages <= 3, "extend the wait ladder");
     if (pending <= 0)
         cp_async_wait<0>();
-    else
+    else if (pending == 1)
         cp_async_wait<1>();
+    else
+        cp_async_wait<2>();
 }
 
 // Gathers the K and V rows of 128-key step `tile` into a stage: sub-tile u (keys 64u..64u+63

@@ -17,6 +17,8 @@
 //   warps 0-3   softmax of stream 0 (thread = TMEM lane = tile row), warps 4-7 stream 1
 //   warp 8      TMA producer: K and V tiles of 128 keys into two 2-stage rings
 //   warp 9      allocates TMEM; one lane issues every tcgen05.mma and commit
+//   warps 10-11 idle after the prologue; with warps 8 and 9 they form the warpgroup that
+//               hands registers to the softmax warpgroups (setmaxnreg)
 // TMEM (512 columns): stream s has S at columns 256s .. 256s+127 (fp32 logits; the bf16
 // probabilities P overwrite its first 64 columns) and O at 256s+128 .. 256s+128+D-1.
 //
@@ -38,7 +40,14 @@ namespace {
 constexpr int kUTile = 128;     // keys per K/V tile
 constexpr int kURows = 128;     // rows per query tile (= TMEM lanes)
 constexpr int kUStages = 2;     // stages of each of the K and V rings
-constexpr int kUThreads = 320;
+constexpr int kUThreads = 384;
+// Registers per thread: at launch (65536 / 384, rounded down to a multiple of 8), and after the
+// split -- the softmax warpgroups hold a whole 128-column row of S; the producer/MMA warpgroup
+// needs few.  The split must not exceed the launch total.
+constexpr int kURegsLaunch = 168;
+constexpr int kURegsSoftmax = 224;
+constexpr int kURegsOther = 56;
+static_assert(2 * 128 * kURegsSoftmax + 128 * kURegsOther <= kUThreads * kURegsLaunch, "register split");
 constexpr float kRescaleBits = 8.f;  // lazy-rescale threshold (base-2 units)
 
 template <int D>
@@ -150,6 +159,8 @@ __global__ void __launch_bounds__(kUThreads, 1)
     const int nstep1 = split_keys ? nt / 2 : nt;
     auto seq_of = [&](int s, int i) { return split_keys ? 2 * i + s : i; };
 
+    if (warp >= 8) {
+        reg_dealloc<kURegsOther>();
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -241,7 +252,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
             mbar_wait(done, 0, a.status);  // nothing of this CTA is left in the tensor core
         }
         __syncwarp();
+    }
     } else {
+        reg_alloc<kURegsSoftmax>();
         // ------------------------------------------------------------ softmax (thread = row)
         const int s = warp >> 2, quarter = warp & 3;
         const int r = quarter * 32 + lane;
@@ -265,7 +278,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tie_regs(x[c]);
             const int j0 = (t_begin + seq_of(s, i)) * kUTile;
-            float mx = -INFINITY;
+            float mx;
             if (j0 + kUTile - 1 > p) {  // tile reaches past this row's position: mask
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
@@ -273,10 +286,18 @@ __global__ void __launch_bounds__(kUThreads, 1)
                     for (int e = 0; e < 32; ++e)
                         if (j0 + 32 * c + e > p) x[c][e] = __float_as_uint(-INFINITY);
             }
+            {  // row max as 8 independent chains (a single chain would serialise 128 dependent ops)
+                float m8[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+                for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(x[0][e]);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(x[c][e]));
+                for (int e = 8; e < 128; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(x[e >> 5][e & 31]));
+#pragma unroll
+                for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                    for (int e = 0; e < w; ++e) m8[e] = fmaxf(m8[e], m8[e + w]);
+                mx = m8[0];
+            }
             mx *= sc;  // base-2 units (sc > 0 keeps the order)
             const bool bump = mx > m_ref + kRescaleBits;
             const float corr = bump ? fast_exp2(m_ref - mx) : 1.f;  // 0 when m_ref = -inf
@@ -297,7 +318,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
                 }
             }
             const float base = m_ref == -INFINITY ? 0.f : m_ref;
-            float sum = 0.f;
+            float sum8[8];  // row sum as 8 independent chains
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
@@ -305,12 +328,16 @@ __global__ void __launch_bounds__(kUThreads, 1)
                 for (int e = 0; e < 16; ++e) {
                     const float p0 = fast_exp2(fmaf(__uint_as_float(x[c][2 * e]), sc, -base));
                     const float p1 = fast_exp2(fmaf(__uint_as_float(x[c][2 * e + 1]), sc, -base));
-                    sum += p0 + p1;
+                    sum8[e & 7] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(tS + 16 * c, pk);
             }
-            l = l * corr + sum;
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) sum8[e] += sum8[e + w];
+            l = l * corr + sum8[0];
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&pfull[s]);
@@ -364,6 +391,11 @@ cudaError_t umma_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUten
     auto kern = umma_attn_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
+    // the register split is sized for exactly kURegsLaunch registers per thread at launch
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kURegsLaunch) return cudaErrorInvalidConfiguration;
     const int split_keys = p.umma_split_keys ? 1 : 0;
     const int QP = split_keys ? p.QB : (p.QB + 1) / 2;
     dim3 grid(p.SU, p.B * p.Hkv * QP);

@@ -264,14 +264,21 @@ __global__ void __launch_bounds__(kSThreads, 1)
                 tie_regs(x[1]);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
+                    // max over the G heads of each query as a tree (independent ops first)
+                    float m[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) m[e] = __uint_as_float(x[hh][e]);
+#pragma unroll
+                    for (int w = G / 2; w > 0; w >>= 1)
+#pragma unroll
+                        for (int qq = 0; qq < 32 / G; ++qq)
+#pragma unroll
+                            for (int g = 0; g < w; ++g) m[qq * G + g] = max_nan(m[qq * G + g], m[qq * G + g + w]);
 #pragma unroll
                     for (int qq = 0; qq < 32 / G; ++qq) {
-                        float m = __uint_as_float(x[hh][qq * G]);
-#pragma unroll
-                        for (int g = 1; g < G; ++g) m = max_nan(m, __uint_as_float(x[hh][qq * G + g]));
                         const int qi = (c0 + 32 * hh) / G + qq;  // query index within these columns
                         if (fast || j <= s_pl[qa0 + qi]) {
-                            const float sv = m * c2;
+                            const float sv = m[qq * G] * c2;
                             nonfinite |= (sv != sv);
                             kp[static_cast<int64_t>(qi) * a.kstride] = score_key(sv);
                         }

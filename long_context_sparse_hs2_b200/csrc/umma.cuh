@@ -133,4 +133,21 @@ __device__ __forceinline__ void tie_regs(uint32_t (&r)[N]) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ------------------------------------------------------------------ register reallocation
+//
+// setmaxnreg moves registers between the warpgroups of a CTA: a warpgroup that lowers its
+// count returns registers to the CTA's pool, one that raises it waits until the pool has them.
+// The pool is what the CTA was launched with (threads x registers per thread at launch), so
+// the counts after the split must add up to no more than that -- checked by the launchers
+// against the kernel's actual register count before every launch.  Every warp of the
+// warpgroup executes the same instruction.
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 }  // namespace hs2
