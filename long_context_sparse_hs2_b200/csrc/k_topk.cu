@@ -300,11 +300,115 @@ __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
 
 // ====================================================================== one CTA per row (many rows)
 //
-// With thousands of selection rows (chunked prefill) one CTA finishes a whole row: it builds
-// the row's histogram in shared memory, finds the threshold bucket with a block scan, then
-// reads the row's keys again (mostly from L2) to write the keys of better buckets and collect
-// the threshold bucket's candidates in shared memory, and radix-selects the exact remainder.
-// No cross-CTA counters or global histograms.
+// With thousands of selection rows (chunked prefill) one CTA finishes a whole row, with no
+// cross-CTA counters or global histograms.  Bucket ranges bracket the threshold:
+//   1. a histogram of a 1/16 sample of the row's keys (one 16-byte group in sixteen) gives
+//      buckets b_lo <= b_hi around the sample's estimate of the keff-th best key, with a
+//      margin of several standard deviations;
+//   2. one pass over all keys writes the keys of buckets < b_lo to the output and collects the
+//      keys of buckets b_lo .. b_hi as candidates in shared memory;
+//   3. if #(bucket < b_lo) <= keff <= #(bucket <= b_hi) and the candidates fit, the selection is
+//      exactly those keys plus the best (keff - #(bucket < b_lo)) candidates by radix select
+//      (a better bucket means a strictly better score);
+//   4. otherwise (an unlucky sample, heavy ties, small pools) the exact two-pass method runs:
+//      full histogram, threshold bucket, emit, radix select.
+// Either way the result is the exact top-keff with ties to the lower index.
+
+namespace {
+
+constexpr int kSampleStride = 16;        // sample one 4-key group in 16
+constexpr int kSampleMinPool = 32768;    // smaller pools go straight to the two-pass method
+
+// Writes the keys of buckets < lo to out (the first `cap` of them) and collects the keys of
+// buckets lo .. hi as candidates in s_cand (the first kSmemCand); counts both in *s_ndef and
+// *s_ncand.  Each thread takes 4 keys per step; a warp with any hit scans its lanes' counts
+// (packed: defs low, candidates high half-word) and reserves slots with one shared atomic per
+// list.  Call from all threads.
+template <int NT>
+__device__ __forceinline__ void emit_bucket_range(const uint32_t* keys, int P, int lo, int hi, int cap, int32_t* out,
+                                                  unsigned long long* s_cand, int* s_ndef, int* s_ncand) {
+    const int lane = threadIdx.x & 31;
+    for (int base = 0; base < P; base += 4 * NT) {  // warp-uniform trip count (shuffles inside)
+        const int j = base + 4 * static_cast<int>(threadIdx.x);
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (j < P) q = __ldcg(reinterpret_cast<const uint4*>(keys + j));
+        const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+        unsigned dmask = 0u, cmask = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int bin = j + e < P ? score_bin(kk[e]) : kHistBins;
+            dmask |= static_cast<unsigned>(bin < lo) << e;
+            cmask |= static_cast<unsigned>(bin >= lo && bin <= hi) << e;
+        }
+        if (!__any_sync(0xffffffffu, (dmask | cmask) != 0u)) continue;
+        const unsigned mine = __popc(dmask) | (__popc(cmask) << 16);  // <= 128 per warp: no carry
+        unsigned incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int bdef = 0, bcnd = 0;
+        if (lane == 31) {
+            if (incl & 0xFFFFu) bdef = atomicAdd(s_ndef, static_cast<int>(incl & 0xFFFFu));
+            if (incl >> 16) bcnd = atomicAdd(s_ncand, static_cast<int>(incl >> 16));
+        }
+        bdef = __shfl_sync(0xffffffffu, bdef, 31);
+        bcnd = __shfl_sync(0xffffffffu, bcnd, 31);
+        const unsigned excl = incl - mine;
+        int od = bdef + static_cast<int>(excl & 0xFFFFu);
+        int oc = bcnd + static_cast<int>(excl >> 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (dmask >> e & 1u) {
+                if (od < cap) out[od] = j + e;
+                ++od;
+            }
+            if (cmask >> e & 1u) {
+                if (oc < kSmemCand) s_cand[oc] = composite(kk[e], j + e);
+                ++oc;
+            }
+        }
+    }
+}
+
+// After a histogram in sh: for each of the two counts c[0], c[1] (>= 1), the smallest bucket b
+// whose cumulative count (buckets 0 .. b) reaches c, and the count below it, into
+// s_bin[i] / s_below[i] (bucket kHistBins - 1 and the count below it if c exceeds the total).
+// Call from all threads (NT of them).
+template <int NT>
+__device__ __forceinline__ void buckets_at_counts(const unsigned* sh, const unsigned (&c)[2], unsigned* s_warp,
+                                                  int* s_bin, int* s_below) {
+    constexpr int PER = kHistBins / NT;
+    const int tid = threadIdx.x;
+    unsigned vals[PER], sum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        vals[i] = sh[tid * PER + i];
+        sum += vals[i];
+    }
+    const unsigned excl = block_exclusive_scan(sum, s_warp);
+    const bool last_thread = tid == NT - 1;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        if (excl < c[k] && c[k] <= excl + sum) {
+            unsigned cum = excl;
+            for (int i = 0; i < PER; ++i) {
+                if (cum + vals[i] >= c[k]) {
+                    s_bin[k] = tid * PER + i;
+                    s_below[k] = static_cast<int>(cum);
+                    break;
+                }
+                cum += vals[i];
+            }
+        } else if (last_thread && c[k] > excl + sum) {  // beyond the total
+            s_bin[k] = kHistBins - 1;
+            s_below[k] = static_cast<int>(excl + sum - vals[PER - 1]);
+        }
+    }
+}
+
+}  // namespace
 
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
@@ -313,16 +417,16 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
     __shared__ unsigned h[256];
     __shared__ unsigned s_small[2];
     __shared__ unsigned s_warp[32];
-    __shared__ int s_b1, s_above, s_ndef, s_ncand, s_count;
+    __shared__ int s_bin[2], s_below[2], s_ndef, s_ncand, s_count, s_nsample;
     static_assert(kHistBins % NT == 0 && NT % 32 == 0, "bins per thread");
     const int64_t row = blockIdx.x;
     const int tid = threadIdx.x;
     pdl_trigger();
     for (int i = tid; i < kHistBins; i += NT) sh[i] = 0u;
     if (tid == 0) {
-        s_ndef = s_ncand = s_count = 0;
-        s_b1 = kHistBins;
-        s_above = -1;
+        s_ndef = s_ncand = s_count = s_nsample = 0;
+        s_bin[0] = s_bin[1] = kHistBins - 1;
+        s_below[0] = s_below[1] = 0;
     }
     const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
     const int kw = a.k + a.W;
@@ -337,9 +441,58 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
         for (int j = tid; j < ri.P; j += NT) out[j] = j;
         return;
     }
-    const uint32_t* keys = a.keys + row * a.kstride;
+    const uint32_t* keys = a.keys + row * a.kstride;  // rows are 256-byte aligned: 16-byte loads
     __syncthreads();
-    // pass 1: histogram (rows are 256-byte aligned: 16-byte loads, 4 keys each)
+
+    if (ri.P >= kSampleMinPool) {
+        // 1. sample histogram
+        int mine = 0;
+        const int groups = (ri.P + 3) / 4;
+        for (int g = tid * kSampleStride; g < groups; g += NT * kSampleStride) {
+            const int j = 4 * g;
+            const uint4 q = __ldcg(reinterpret_cast<const uint4*>(keys + j));
+            const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (j + e < ri.P) {
+                    atomicAdd(&sh[score_bin(kk[e])], 1u);
+                    ++mine;
+                }
+        }
+        if (mine) atomicAdd(&s_nsample, mine);
+        __syncthreads();
+        const float ns = static_cast<float>(s_nsample);
+        const float r = static_cast<float>(ri.keff) * ns / static_cast<float>(ri.P);  // expected sample rank
+        const float margin = 4.f * sqrtf(r) + 16.f;
+        const unsigned c[2] = {static_cast<unsigned>(fmaxf(r - margin, 0.f)) + 1u,
+                               static_cast<unsigned>(fminf(r + margin, ns)) + 1u};
+        buckets_at_counts<NT>(sh, c, s_warp, s_bin, s_below);
+        __syncthreads();
+        // 2. one pass: buckets < lo out, lo .. hi candidates
+        const int lo = s_bin[0], hi = s_bin[1];
+        emit_bucket_range<NT>(keys, ri.P, lo, hi, ri.keff, out, s_cand, &s_ndef, &s_ncand);
+        __syncthreads();
+        // 3. bracketed?
+        const int ndef = s_ndef, ncand = s_ncand;
+        if (ndef <= ri.keff && ri.keff <= ndef + ncand && ncand <= kSmemCand) {
+            const unsigned need = static_cast<unsigned>(ri.keff - ndef);
+            if (need > 0) {
+                const SmemSource src{s_cand, ncand};
+                emit_at_least(src, radix_threshold(src, need, h, s_small), need, out + ndef, &s_count);
+            }
+            return;
+        }
+        // 4. not bracketed: start over with the exact two-pass method
+        for (int i = tid; i < kHistBins; i += NT) sh[i] = 0u;
+        if (tid == 0) {
+            s_ndef = s_ncand = 0;
+            s_bin[0] = s_bin[1] = kHistBins - 1;
+            s_below[0] = s_below[1] = 0;
+        }
+        __syncthreads();
+    }
+
+    // exact two-pass method: full histogram
     for (int base = 0; base < ri.P; base += 4 * NT) {
         const int j = base + 4 * tid;
         if (j < ri.P) {
@@ -352,77 +505,14 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
     }
     __syncthreads();
     {
-        constexpr int PER = kHistBins / NT;
-        unsigned vals[PER], sum = 0;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            vals[i] = sh[tid * PER + i];
-            sum += vals[i];
-        }
-        const unsigned excl = block_exclusive_scan(sum, s_warp);
-        const unsigned need = static_cast<unsigned>(ri.keff);
-        if (excl < need && need <= excl + sum) {
-            unsigned cum = excl;
-            for (int i = 0; i < PER; ++i) {
-                if (cum + vals[i] >= need) {
-                    s_b1 = tid * PER + i;
-                    s_above = static_cast<int>(cum);
-                    break;
-                }
-                cum += vals[i];
-            }
-        }
+        const unsigned c[2] = {static_cast<unsigned>(ri.keff), static_cast<unsigned>(ri.keff)};
+        buckets_at_counts<NT>(sh, c, s_warp, s_bin, s_below);
     }
     __syncthreads();
-    const int b1 = s_b1, above = s_above;
+    const int b1 = s_bin[0], above = s_below[0];
     if (above < 0 || above >= ri.keff) return;  // cannot happen for a consistent histogram
-    // pass 2: keys of better buckets go straight out, the threshold bucket's are candidates.
-    // Each thread has 4 keys; a warp with any hit scans its per-lane counts (packed: defs in the
-    // low, candidates in the high half-word) and reserves its slots with one shared-memory
-    // atomic per list.
-    const int lane = tid & 31;
-    for (int base = 0; base < ri.P; base += 4 * NT) {  // warp-uniform trip count (shuffles inside)
-        const int j = base + 4 * tid;
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (j < ri.P) q = __ldcg(reinterpret_cast<const uint4*>(keys + j));
-        const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
-        unsigned dmask = 0u, cmask = 0u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int bin = j + e < ri.P ? score_bin(kk[e]) : kHistBins;
-            dmask |= static_cast<unsigned>(bin < b1) << e;
-            cmask |= static_cast<unsigned>(bin == b1) << e;
-        }
-        if (!__any_sync(0xffffffffu, (dmask | cmask) != 0u)) continue;
-        const unsigned mine = __popc(dmask) | (__popc(cmask) << 16);  // <= 128 per warp: no carry
-        unsigned incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        int bdef = 0, bcnd = 0;
-        if (lane == 31) {
-            if (incl & 0xFFFFu) bdef = atomicAdd(&s_ndef, static_cast<int>(incl & 0xFFFFu));
-            if (incl >> 16) bcnd = atomicAdd(&s_ncand, static_cast<int>(incl >> 16));
-        }
-        bdef = __shfl_sync(0xffffffffu, bdef, 31);
-        bcnd = __shfl_sync(0xffffffffu, bcnd, 31);
-        const unsigned excl = incl - mine;
-        int od = bdef + static_cast<int>(excl & 0xFFFFu);
-        int oc = bcnd + static_cast<int>(excl >> 16);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (dmask >> e & 1u) {
-                if (od < above) out[od] = j + e;
-                ++od;
-            }
-            if (cmask >> e & 1u) {
-                if (oc < kSmemCand) s_cand[oc] = composite(kk[e], j + e);
-                ++oc;
-            }
-        }
-    }
+    // keys of better buckets go straight out, the threshold bucket's are candidates
+    emit_bucket_range<NT>(keys, ri.P, b1, b1, above, out, s_cand, &s_ndef, &s_ncand);
     __syncthreads();
     const unsigned need = static_cast<unsigned>(ri.keff - above);
     const int ncand = s_ncand;

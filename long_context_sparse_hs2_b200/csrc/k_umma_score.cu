@@ -15,11 +15,11 @@
 // per-row block (-u split into three bf16 parts whose sum is u to about 24 bits), so TMEM
 // already holds x - u and the epilogue is a max over heads and one scale per (query, key).
 //
-// Roles (320 threads): warps 0-3 and 4-7 are two epilogue warpgroups that split the columns
-// of every tile between them (one query tile each, or half of one); two TMEM accumulators
-// (256 columns each) let the MMA of tile i + 1 run during the epilogue of tile i; warp 8
-// streams K tiles of 128 keys (3-stage TMA ring); warp 9 allocates TMEM and one of its lanes
-// issues the MMAs.  Every wait is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains
+// Roles (576 threads): warps 0-15 are four epilogue warpgroups that split the columns of
+// every tile between them (a quarter each); two TMEM accumulators (256 columns each) let the
+// MMA of tile i + 1 run during the epilogue of tile i, and a warpgroup hands its accumulator
+// back as soon as it has read its columns; warp 16 streams K tiles of 128 keys (3-stage TMA
+// ring); warp 17 allocates TMEM and one of its lanes issues the MMAs.  Every wait is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains
 // and exits.
 #include "attn_sweep.cuh"
 #include "umma.cuh"
@@ -31,7 +31,9 @@ namespace {
 constexpr int kSTile = 128;      // keys per K tile (= TMEM lanes = M)
 constexpr int kURowsPerTile = 128;  // query-head rows per query tile
 constexpr int kSStages = 3;
-constexpr int kSThreads = 320;
+constexpr int kSEpiWarps = 16;  // four epilogue warpgroups
+constexpr int kSProducer = kSEpiWarps, kSMma = kSEpiWarps + 1;
+constexpr int kSThreads = (kSEpiWarps + 2) * 32;
 constexpr int kSMaxCols = 256;   // query-head rows per CTA (two query tiles)
 
 template <int D>
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < L::kNumBars; ++i) {
             const bool is_tfree = i >= 2 * kSStages + 2 && i < 2 * kSStages + 4;
-            mbar_init(&bars[i], is_tfree ? 2 * kSTile : 1);  // tfree: one arrival per epilogue thread
+            mbar_init(&bars[i], is_tfree ? kSEpiWarps * 32 : 1);  // tfree: one arrival per epilogue thread
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
         *reinterpret_cast<uint4*>(smem + L::kQcOff + R * 128 + ((c ^ (R & 7)) << 4)) = v;
     }
     fence_async_smem();
-    if (warp == 9) {
+    if (warp == kSMma) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
     }
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     const int nt = t_end - t_begin;
 
     bool nonfinite = false;
-    if (warp == 8) {
+    if (warp == kSProducer) {
         // ------------------------------------------------------------ TMA producer (K only)
         if (lane == 0) {
             const uint64_t pol = a.stream_kv ? l2_evict_first() : l2_evict_normal();
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == kSMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(kSTile, ncols, false);
@@ -232,9 +234,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue (thread = key)
-        const int w = warp >> 2, quarter = warp & 3;
+        const int w = warp >> 2, quarter = warp & 3;  // warpgroup, TMEM lane quarter
         const int r = quarter * 32 + lane;
-        const int wcols = ncols / 2;           // columns of this warpgroup: one query tile, or half of one
+        const int wcols = ncols / (kSEpiWarps / 4);  // columns of this warpgroup: a quarter of the tile
         const int col0 = w * wcols;
         const int s = col0 / kURowsPerTile;    // query tile of these columns
         const int qa0 = col0 / G, nqw = wcols / G;
@@ -255,44 +257,52 @@ __global__ void __launch_bounds__(kSThreads, 1)
             const int j = jt + r;
             const bool fast = jt + kSTile - 1 <= plmin;  // every query of these columns takes every key
             uint32_t* kp = a.keys + row0 * a.kstride + j;
-            for (int c0 = 0; c0 < wcols; c0 += 64) {
-                uint32_t x[2][32];
-                tmem_ld32(tbase + 256 * buf + c0, x[0]);
-                tmem_ld32(tbase + 256 * buf + c0 + 32, x[1]);
-                tmem_wait_ld();
-                tie_regs(x[0]);
-                tie_regs(x[1]);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    // max over the G heads of each query as a tree (independent ops first)
-                    float m[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) m[e] = __uint_as_float(x[hh][e]);
-#pragma unroll
-                    for (int w = G / 2; w > 0; w >>= 1)
-#pragma unroll
-                        for (int qq = 0; qq < 32 / G; ++qq)
-#pragma unroll
-                            for (int g = 0; g < w; ++g) m[qq * G + g] = max_nan(m[qq * G + g], m[qq * G + g + w]);
-#pragma unroll
-                    for (int qq = 0; qq < 32 / G; ++qq) {
-                        const int qi = (c0 + 32 * hh) / G + qq;  // query index within these columns
-                        if (fast || j <= s_pl[qa0 + qi]) {
-                            const float sv = m[qq * G] * c2;
-                            nonfinite |= (sv != sv);
-                            kp[static_cast<int64_t>(qi) * a.kstride] = score_key(sv);
-                        }
-                    }
-                }
-            }
+            // read all of this warpgroup's columns, then hand the accumulator back to the MMA
+            // before the max / key conversion / stores
+            uint32_t x[2][32];
+            tmem_ld32(tbase + 256 * buf, x[0]);
+            if (wcols > 32) tmem_ld32(tbase + 256 * buf + 32, x[1]);
+            tmem_wait_ld();
+            tie_regs(x[0]);
+            tie_regs(x[1]);
             tc_fence_before();
             mbar_arrive(&tfree[buf]);
+#pragma unroll
+            for (int cq = 0; cq < 2; ++cq) {
+                if (32 * cq >= wcols) break;
+                // max over the G heads of each query as a tree (independent ops first)
+                float m[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) m[e] = __uint_as_float(x[cq][e]);
+#pragma unroll
+                for (int w2 = G / 2; w2 > 0; w2 >>= 1)
+#pragma unroll
+                    for (int qq = 0; qq < 32 / G; ++qq)
+#pragma unroll
+                        for (int g = 0; g < w2; ++g) m[qq * G + g] = max_nan(m[qq * G + g], m[qq * G + g + w2]);
+                uint32_t key[32 / G];
+#pragma unroll
+                for (int qq = 0; qq < 32 / G; ++qq) {
+                    const float sv = m[qq * G] * c2;
+                    nonfinite |= (sv != sv);
+                    key[qq] = score_key(sv);
+                }
+                uint32_t* kq = kp + static_cast<int64_t>((32 * cq) / G) * a.kstride;
+                if (fast) {  // every query of these columns takes this key
+#pragma unroll
+                    for (int qq = 0; qq < 32 / G; ++qq) __stcs(kq + static_cast<int64_t>(qq) * a.kstride, key[qq]);
+                } else {
+#pragma unroll
+                    for (int qq = 0; qq < 32 / G; ++qq)
+                        if (j <= s_pl[qa0 + (32 * cq) / G + qq]) __stcs(kq + static_cast<int64_t>(qq) * a.kstride, key[qq]);
+                }
+            }
         }
     }
 
     tc_fence_before();
     if (__syncthreads_or(nonfinite) && tid == 0) set_status(a.status, HS2_DEV_NONFINITE);
-    if (warp == 9) {
+    if (warp == kSMma) {
         tc_fence_after();
         tmem_dealloc(tm, 512);
     }

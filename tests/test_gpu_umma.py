@@ -134,3 +134,29 @@ def test_many_rows_all_scores_equal():
     ref = compare_step(inp, res)
     for (b, h, t), r in ref.items():
         np.testing.assert_array_equal(np.sort(res["idx"][b, h, t][:res["cnt"][b, h, t]]), r.selected)
+
+
+def test_many_rows_large_pools_sample_bracket():
+    # pools >= 32768 keys: the row top-k brackets the threshold from a 1/16 sample and selects
+    # in one pass; checked on sampled rows against the oracle and on every row's invariants
+    from tests.test_gpu_parity import compare_step, run_step
+    from tests.test_gpu_workloads import check_all_rows
+
+    inp = make_inputs(1, 8, 1, 128, 40000, 600, 2048, 128, seed=23, needles=32)
+    res = run_step(inp)
+    check_all_rows(inp, res["idx"], res["cnt"])
+    compare_step(inp, res, rows=[(0, 0, t) for t in (0, 1, 77, 300, 301, 598, 599)])
+
+
+def test_many_rows_large_pools_all_ties_fall_back():
+    # every score equal: the sample cannot bracket the threshold within shared memory, so the
+    # exact two-pass method runs (and re-scans the keys for the tied bucket)
+    from tests.test_gpu_parity import compare_step, run_step
+
+    inp = make_inputs(1, 8, 1, 128, 40000, 600, 500, 64, seed=24)
+    inp.Qf = np.zeros_like(inp.Qf)
+    res = run_step(inp)
+    rows = [(0, 0, t) for t in (0, 299, 599)]
+    ref = compare_step(inp, res, rows=rows)
+    for (b, h, t), r in ref.items():
+        np.testing.assert_array_equal(np.sort(res["idx"][b, h, t][:res["cnt"][b, h, t]]), r.selected)
