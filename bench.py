@@ -76,17 +76,60 @@ def byte_model(w):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs.
+
+    NVML is polled every millisecond from a background thread (a decode step is ~0.1 ms, so
+    nvidia-smi's 100 ms polling would miss a short timed region entirely); one sample is also
+    taken on entry and on exit.  Without NVML it falls back to `nvidia-smi -lms 100`.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvmlClocksEventReason*)
+    REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                   0x40: "hw_thermal_slowdown"}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.nvml = None
+        self.samples = []
+        self.lines = []
+
+    # -- NVML path
+    def _nvml_sample(self):
+        nv, h = self.nvml, self.handle
+        try:
+            clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.samples.append((float(clk), int(get_reasons(h))))
+        except Exception:
+            pass
+
+    def _nvml_loop(self):
+        while True:
+            self._nvml_sample()
+            if self.stop.wait(0.001):
+                break
 
     def __enter__(self):
+        try:
+            import pynvml
+            import threading
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self._nvml_sample()
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -96,7 +139,15 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.nvml is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            self._nvml_sample()
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            return
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -108,8 +159,15 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], None, set()
+        if self.samples:
+            for clk, bits in self.samples:
+                sm.append(clk)
+                for bit, nm in self.REASON_BITS.items():
+                    if bits & bit:
+                        reasons.add(nm)
+            mx = self.max_mhz
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -123,7 +181,8 @@ class ClockSampler:
                     reasons.add(nm)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvml" if self.samples else "nvidia-smi"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm

@@ -24,7 +24,8 @@ Recipe (stated once here, repeated in the design notes):
   ``pos[b, t] = N - T + t``.
 
 The named workloads are the five shapes the long-context decode and chunked
-prefill benchmarks use (the 1M-token decode appears twice, at T=1 and T=16).
+prefill benchmarks use (the 1M-token decode appears twice, at T=1 and T=16), plus
+a reduced chunked-prefill shape for profiler captures.
 The pages run no public benchmark for this step; these needle-in-noise inputs
 stand in for long-context retrieval traffic.
 """
@@ -71,6 +72,10 @@ WORKLOADS = {
                       seed=4, needles=512),
     "1m_t16": Workload("1m_t16", B=1, Hq=32, Hkv=4, d=128, N=1048576, T=16, k=8192, W=1024,
                        seed=4, needles=512),
+    # the chunked-prefill shape at a quarter of the context and of the chunk: small enough for
+    # multi-pass profiler captures of the prefill kernels (K/V 64 MiB, score keys 512 MiB)
+    "prefill_32k": Workload("prefill_32k", B=1, Hq=32, Hkv=4, d=128, N=32768, T=1024, k=2048, W=128,
+                            seed=3, needles=64),
 }
 
 
