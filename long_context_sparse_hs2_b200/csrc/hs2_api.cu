@@ -100,10 +100,11 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
               (static_cast<int64_t>(x.k) + x.W + P.S1 - 1) / P.S1 <= kFusedMaxSlice;
 
     // sparse attention: about one CTA per SM, each gathering C4 keys (a multiple of 64, <= 1024)
+    // -- or, with many rows, a whole row (up to kSparseMaxC4 keys) per CTA, no split partials.
+    // (One 128-key step per CTA at two CTAs per SM measured slower for the decode shapes.)
     const int64_t kw = static_cast<int64_t>(x.k) + x.W;
     const int64_t s4_target = std::max<int64_t>(1, kSMs / rows_kv);
     const int64_t c4 = ((std::max<int64_t>(1, (kw + s4_target - 1) / s4_target) + 63) / 64) * 64;
-    // with many rows every CTA takes a whole row (up to kSparseMaxC4 keys): no split partials
     const int64_t c4_cap = rows_kv >= 2 * kSMs ? kSparseMaxC4 : 1024;
     P.C4 = static_cast<int>(std::min<int64_t>(c4_cap, std::max<int64_t>(64, c4)));
     P.S4 = static_cast<int>(std::max<int64_t>(1, (kw + P.C4 - 1) / P.C4));

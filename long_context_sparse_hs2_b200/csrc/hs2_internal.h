@@ -90,6 +90,7 @@ struct SparseArgs {
     const int32_t* cnt;    // [rows_kv]
     int B, Hq, Hkv, T, N, G, kw;  // kw = k + W (row stride of idx)
     int C4, S4;
+    int stages;            // gather ring depth (set by the launcher)
     float scale_log2;
     float2* part_ml;       // [S4][rows_q]
     float* part_acc;       // [S4][rows_q][D]

@@ -15,6 +15,8 @@
 // four 64-key tiles in flight -- and runs the shared warp attention core.  The row's last
 // CTA to finish (a completion counter; nothing waits) merges the S4 split partials into
 // O_sparse and LSE_sparse.
+#include <algorithm>
+
 #include "attn_core.cuh"
 #include "combine.cuh"
 #include "hs2_internal.h"
@@ -27,21 +29,28 @@ constexpr int kSparseWarps = 8;
 constexpr int kSparseThreads = kSparseWarps * 32;
 constexpr int kSparseTile = 2 * kKeyTile;  // keys per pipeline step: two 64-key sub-tiles
 
-constexpr int kSparseStages = 3;
+constexpr int kSparseMaxStages = 3;  // ring depth for long rows; short rows use fewer (less smem)
 
 template <int D>
 struct SparseSmem {
     static constexpr int kTileBytes = kKeyTile * D * 2;    // one 64-key sub-tile of K (or V)
     static constexpr int kSubBytes = 2 * kTileBytes;       // K + V of one sub-tile
     static constexpr int kStageBytes = 2 * kSubBytes;      // two sub-tiles = one 128-key step
-    static constexpr int kRingBytes = kSparseStages * kStageBytes;
-    static constexpr int kIdxOff = kRingBytes;
-    static constexpr int bytes(int C4) { return kIdxOff + (C4 + kSparseTile) * 4 + 16 + 1024; }
+    // After the main loop the ring is reused as scratch: the warps' softmax states are merged
+    // there (merge_states) and the row's last CTA keeps its combine weights there; the region
+    // before the index list is at least as large as either.
+    static constexpr int kMergeBytes = merge_floats<D, kSparseWarps>() * 4;
+    static constexpr int kCombineBytes = (8192 / 2 + 1 + 16) * 8;  // G * S4 <= 8192 weights, then G <= 16 (m, l)
+    static constexpr int kScratchBytes = kMergeBytes > kCombineBytes ? kMergeBytes : kCombineBytes;
+    static constexpr int idx_off(int stages) {
+        return stages * kStageBytes > kScratchBytes ? stages * kStageBytes : kScratchBytes;
+    }
+    static constexpr int bytes(int stages, int C4) { return idx_off(stages) + (C4 + kSparseTile) * 4 + 16 + 1024; }
 };
 
 // Wait until at most `pending` of this thread's cp.async groups are still in flight.
 __device__ __forceinline__ void cp_async_wait_upto(int pending) {
-    static_assert(kSparseStages <= 3, "extend the wait ladder");
+    static_assert(kSparseMaxStages <= 3, "extend the wait ladder");
     if (pending <= 0)
         cp_async_wait<0>();
     else if (pending == 1)
@@ -95,13 +104,16 @@ __device__ __forceinline__ void finish_row(const SparseArgs& a, int row, int64_t
 
 }  // namespace
 
-template <int D>
-__global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const SparseArgs a) {
+// MINB: CTAs per SM the register allocation must allow (2 for one-step CTAs, whose ring is a
+// single 64 KB stage; 1 for the deep-ring variant, which also gets the registers to avoid spills).
+template <int D, int MINB>
+__global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const SparseArgs a) {
     using L = SparseSmem<D>;
     constexpr int KW = 16;  // keys per warp per step: warps 0-3 take sub-tile 0, warps 4-7 sub-tile 1
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int* s_idx = reinterpret_cast<int*>(smem + L::kIdxOff);
+    const int stages = a.stages;  // ring depth: min(3, 128-key steps of a CTA)
+    int* s_idx = reinterpret_cast<int*>(smem + L::idx_off(stages));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x;
@@ -149,7 +161,7 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     if (__syncthreads_or(bad) && tid == 0) set_status(a.status, HS2_DEV_BAD_INDEX);
 
     const int64_t kv_base = static_cast<int64_t>(bh) * a.N;
-    const int prime = min(ntl, kSparseStages);
+    const int prime = min(ntl, stages);
     for (int i = 0; i < prime; ++i) {
         gather_tile<D>(a, s_idx, i, smem + i * L::kStageBytes, kv_base);
         cp_async_commit();
@@ -166,9 +178,9 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     const int sub = warp >> 2;
     const int key0 = (warp & 3) * KW;
     for (int i = 0; i < ntl; ++i) {
-        cp_async_wait_upto(min(ntl, i + kSparseStages) - (i + 1));  // step i has landed
+        cp_async_wait_upto(min(ntl, i + stages) - (i + 1));  // step i has landed
         __syncthreads();
-        const int stage = i % kSparseStages;
+        const int stage = i % stages;
         const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes + sub * L::kSubBytes);
         const uint32_t vbase = kbase + L::kTileBytes;
         float sc[KW / 8][4];
@@ -183,8 +195,8 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
             }
         st.template update<KW>(sc, vbase, key0);
         __syncthreads();  // everyone is done with this stage before it is refilled
-        if (i + kSparseStages < ntl) {
-            gather_tile<D>(a, s_idx, i + kSparseStages, smem + stage * L::kStageBytes, kv_base);
+        if (i + stages < ntl) {
+            gather_tile<D>(a, s_idx, i + stages, smem + stage * L::kStageBytes, kv_base);
             cp_async_commit();
         }
     }
@@ -196,22 +208,23 @@ __global__ void __launch_bounds__(kSparseThreads) sparse_attn_kernel(const Spars
     finish_row<D>(a, row, out_rows_q_base(a, b, h, t), smem);
 }
 
-cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st) {
-    dim3 grid(p.S4, static_cast<unsigned>(p.rows_kv));
-    if (p.d == 128) {
-        const int bytes = SparseSmem<128>::bytes(p.C4);
-        cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(sparse_attn_kernel<128>, grid, dim3(kSparseThreads), bytes, st, a);
-        trace_mark("sparse_attn_combine", st);
-        return e;
-    }
-    const int bytes = SparseSmem<64>::bytes(p.C4);
-    cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+template <int D, int MINB>
+cudaError_t sparse_variant(const Plan& p, const SparseArgs& x, cudaStream_t st) {
+    auto kern = sparse_attn_kernel<D, MINB>;
+    const int bytes = SparseSmem<D>::bytes(x.stages, p.C4);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(sparse_attn_kernel<64>, grid, dim3(kSparseThreads), bytes, st, a);
+    e = launch_pdl(kern, dim3(p.S4, static_cast<unsigned>(p.rows_kv)), dim3(kSparseThreads), bytes, st, x);
     trace_mark("sparse_attn_combine", st);
     return e;
+}
+
+cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st) {
+    SparseArgs x = a;
+    x.stages = std::min(kSparseMaxStages, (p.C4 + kSparseTile - 1) / kSparseTile);
+    const bool one_step = x.stages == 1;
+    if (p.d == 128) return one_step ? sparse_variant<128, 2>(p, x, st) : sparse_variant<128, 1>(p, x, st);
+    return one_step ? sparse_variant<64, 2>(p, x, st) : sparse_variant<64, 1>(p, x, st);
 }
 
 }  // namespace hs2
