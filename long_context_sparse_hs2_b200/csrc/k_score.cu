@@ -9,7 +9,7 @@
 // the score open; this library fixes it to the GQA-max log-softmax.
 //
 // Grid (x, y = selection row):
-//   x < nscore: one 4096-key chunk of the row's pool.  The CTA merges the G heads' LSE from
+//   x < nscore: one kTopkChunk-key chunk of the row's pool.  The CTA merges the G heads' LSE from
 //     the split partials, forms every key's score (base-2 units, NaN-propagating max), writes
 //     the order-preserving key, and bins it in a shared-memory histogram that is added to
 //     the row's global histogram; the row's last CTA finds the threshold bucket.
