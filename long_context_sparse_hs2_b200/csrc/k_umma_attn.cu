@@ -286,17 +286,18 @@ __global__ void __launch_bounds__(kUThreads, 1)
                     for (int e = 0; e < 32; ++e)
                         if (j0 + 32 * c + e > p) x[c][e] = __float_as_uint(-INFINITY);
             }
-            {  // row max as 8 independent chains (a single chain would serialise 128 dependent ops)
+            {  // row max: 8 independent chains of three-input maxes (a single chain would
+               // serialise 127 dependent ops)
                 float m8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(x[0][e]);
+                for (int u = 0; u < 8; ++u) m8[u] = fmaxf(__uint_as_float(x[0][u]), __uint_as_float(x[0][8 + u]));
 #pragma unroll
-                for (int e = 8; e < 128; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(x[e >> 5][e & 31]));
+                for (int e = 16; e < 128; e += 16)  // values e .. e + 15: two per chain
 #pragma unroll
-                for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                    for (int e = 0; e < w; ++e) m8[e] = fmaxf(m8[e], m8[e + w]);
-                mx = m8[0];
+                    for (int u = 0; u < 8; ++u)
+                        m8[u] = max3f(m8[u], __uint_as_float(x[(e + u) >> 5][(e + u) & 31]),
+                                      __uint_as_float(x[(e + 8 + u) >> 5][(e + 8 + u) & 31]));
+                mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
             }
             mx *= sc;  // base-2 units (sc > 0 keeps the order)
             const bool bump = mx > m_ref + kRescaleBits;
@@ -318,26 +319,34 @@ __global__ void __launch_bounds__(kUThreads, 1)
                 }
             }
             const float base = m_ref == -INFINITY ? 0.f : m_ref;
-            float sum8[8];  // row sum as 8 independent chains
+            // exponents and the row sum on packed pairs: x * sc - base by one f32x2 FMA per pair,
+            // the sum as 4 independent chains of f32x2 adds (8 scalar chains)
+            const uint64_t sc2 = f2_pack(sc, sc), nb2 = f2_pack(-base, -base);
+            uint64_t sum4[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+            for (int e = 0; e < 4; ++e) sum4[e] = f2_pack(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(x[c][2 * e]), sc, -base));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(x[c][2 * e + 1]), sc, -base));
-                    sum8[e & 7] += p0 + p1;
+                    float a0, a1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(x[c][2 * e]), __uint_as_float(x[c][2 * e + 1])), sc2, nb2),
+                              a0, a1);
+                    const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+                    sum4[e & 3] = f2_add(sum4[e & 3], f2_pack(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(tS + 16 * c, pk);
             }
-#pragma unroll
-            for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                for (int e = 0; e < w; ++e) sum8[e] += sum8[e + w];
-            l = l * corr + sum8[0];
+            float rs;
+            {
+                const uint64_t s2 = f2_add(f2_add(sum4[0], sum4[1]), f2_add(sum4[2], sum4[3]));
+                float s_lo, s_hi;
+                f2_unpack(s2, s_lo, s_hi);
+                rs = s_lo + s_hi;
+            }
+            l = l * corr + rs;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&pfull[s]);

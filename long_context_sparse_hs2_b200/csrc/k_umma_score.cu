@@ -58,6 +58,30 @@ __device__ __forceinline__ float max_nan(float a, float b) {
     asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
     return r;
 }
+__device__ __forceinline__ float max_nan3(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// NaN-propagating max of the G values v[0 .. G-1] (three-input maxes)
+template <int G>
+__device__ __forceinline__ float head_max(const float* v) {
+    if constexpr (G == 1) {
+        return v[0];
+    } else if constexpr (G == 2) {
+        return max_nan(v[0], v[1]);
+    } else if constexpr (G == 4) {
+        return max_nan(max_nan3(v[0], v[1], v[2]), v[3]);
+    } else if constexpr (G == 8) {
+        return max_nan3(max_nan3(v[0], v[1], v[2]), max_nan3(v[3], v[4], v[5]), max_nan(v[6], v[7]));
+    } else {
+        static_assert(G == 16, "G in {1, 2, 4, 8, 16}");
+        const float a = max_nan3(max_nan3(v[0], v[1], v[2]), max_nan3(v[3], v[4], v[5]), max_nan3(v[6], v[7], v[8]));
+        const float b = max_nan3(max_nan3(v[9], v[10], v[11]), max_nan3(v[12], v[13], v[14]), v[15]);
+        return max_nan(a, b);
+    }
+}
 
 __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
     uint32_t r;
@@ -270,20 +294,14 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
             for (int cq = 0; cq < 2; ++cq) {
                 if (32 * cq >= wcols) break;
-                // max over the G heads of each query as a tree (independent ops first)
+                // max over the G heads of each query (three-input maxes, independent queries)
                 float m[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) m[e] = __uint_as_float(x[cq][e]);
-#pragma unroll
-                for (int w2 = G / 2; w2 > 0; w2 >>= 1)
-#pragma unroll
-                    for (int qq = 0; qq < 32 / G; ++qq)
-#pragma unroll
-                        for (int g = 0; g < w2; ++g) m[qq * G + g] = max_nan(m[qq * G + g], m[qq * G + g + w2]);
                 uint32_t key[32 / G];
 #pragma unroll
                 for (int qq = 0; qq < 32 / G; ++qq) {
-                    const float sv = m[qq * G] * c2;
+                    const float sv = head_max<G>(m + qq * G) * c2;
                     nonfinite |= (sv != sv);
                     key[qq] = score_key(sv);
                 }
