@@ -128,12 +128,14 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, c
                            void* ws, size_t ws_bytes, void* stream);
 
 /* The whole hybrid step: hs2_full_attn, hs2_select and hs2_sparse_attn in order on one
- * stream, sharing intermediates through ws.  With one query per batch row (T = 1) and the
- * environment variable HS2_FUSED_DECODE=1 the step runs as a single cooperative kernel when
- * its grid fits on the device (same results up to rounding order; the workspace size depends
- * on the setting, so query hs2_workspace_size under the same environment); when T*G <= 16 the
- * full-attention pass
- * also keeps its logits so the selection does not read K a second time). */
+ * stream, sharing intermediates through ws.  When T*G <= 16 the full-attention pass keeps its
+ * logits so the selection does not read K a second time; when T*G > 64 (128-row query tiles:
+ * chunked prefill, multi-query decode) the full-attention and score sweeps run on the tcgen05
+ * tensor cores.  Two environment variables change the execution plan (results are the same up
+ * to rounding order; the workspace size depends on them, so query hs2_workspace_size under the
+ * same environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles, and with one
+ * query per batch row (T = 1) HS2_FUSED_DECODE=1 runs the step as a single cooperative kernel
+ * when its grid fits on the device. */
 HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
                     const void* K, const void* V, const int32_t* pos,
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,
