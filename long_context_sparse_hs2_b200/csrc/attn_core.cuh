@@ -71,9 +71,16 @@ struct OnlineSoftmax {
     }
 
     // Fold in a slice of base-2 logits s (already masked with -inf); V from the swizzled tile at vbase.
+    // The reference max m is raised only when the slice's max exceeds it by more than
+    // kLazyRescale (base 2): exponentials stay <= 2^kLazyRescale, and the O rescale (D/4
+    // multiplies per lane) is skipped by the whole warp unless some row raised its max.  Exact:
+    // l and O always share the same reference m.
     template <int KW>
     __device__ __forceinline__ void update(float (&s)[KW / 8][4], uint32_t vbase, int key0) {
+        constexpr float kLazyRescale = 8.f;
         const int lane = threadIdx.x & 31;
+        float corr[2];
+        bool bumped = false;
 #pragma unroll
         for (int ri = 0; ri < 2; ++ri) {
             float mx = -INFINITY;
@@ -81,9 +88,11 @@ struct OnlineSoftmax {
             for (int n = 0; n < KW / 8; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * ri], s[n][2 * ri + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m[ri], mx);
+            const bool bump = mx > m[ri] + kLazyRescale;  // false while both are -inf
+            const float m_new = bump ? mx : m[ri];
             const float base = (m_new == -INFINITY) ? 0.f : m_new;
-            const float corr = fast_exp2(m[ri] - base);
+            corr[ri] = bump ? fast_exp2(m[ri] - base) : 1.f;  // 0 when m was -inf
+            bumped |= bump;
             float sum = 0.f;
 #pragma unroll
             for (int n = 0; n < KW / 8; ++n) {
@@ -91,12 +100,16 @@ struct OnlineSoftmax {
                 s[n][2 * ri + 1] = fast_exp2(s[n][2 * ri + 1] - base);
                 sum += s[n][2 * ri] + s[n][2 * ri + 1];
             }
-            l[ri] = l[ri] * corr + sum;
+            l[ri] = l[ri] * corr[ri] + sum;
             m[ri] = m_new;
+        }
+        if (__any_sync(0xffffffffu, bumped)) {
 #pragma unroll
             for (int n = 0; n < D / 8; ++n) {
-                o[n][2 * ri] *= corr;
-                o[n][2 * ri + 1] *= corr;
+                o[n][0] *= corr[0];
+                o[n][1] *= corr[0];
+                o[n][2] *= corr[1];
+                o[n][3] *= corr[1];
             }
         }
         // O += P V

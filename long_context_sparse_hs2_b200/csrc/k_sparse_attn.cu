@@ -60,24 +60,26 @@ __device__ __forceinline__ void cp_async_wait_upto(int pending) {
 }
 
 // Gathers the K and V rows of 128-key step `tile` into a stage: sub-tile u (keys 64u..64u+63
-// of the step) at u * kSubBytes, K then V, each in the swizzled 64-key tile layout.
+// of the step) at u * kSubBytes, K then V, each in the swizzled 64-key tile layout.  Thread t
+// copies 16-byte chunk t mod (D/8) of rows t / (D/8), + 256/(D/8), ... of both sub-tiles, K and
+// V alike: one index load and one address per row for two copies.
 template <int D>
 __device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_idx, int tile, uint8_t* stage,
                                             int64_t kv_base) {
-    constexpr int CH = D / 8;                 // 16-byte chunks per row
-    constexpr int PER_T = kKeyTile * CH;      // chunks per tensor per sub-tile
-    for (int ch = threadIdx.x; ch < 4 * PER_T; ch += kSparseThreads) {
-        const int sub = ch / (2 * PER_T);
-        const int rem2 = ch - sub * 2 * PER_T;
-        const int tensor = rem2 / PER_T;
-        const int rem = rem2 - tensor * PER_T;
-        const int r = rem / CH, c16 = rem - r * CH;
-        const int j = s_idx[tile * kSparseTile + sub * kKeyTile + r];
-        const uint16_t* base = tensor ? a.V : a.K;
-        const uint16_t* src = base + (kv_base + (j >= 0 ? j : 0)) * D + c16 * 8;
-        cp_async16(stage + sub * SparseSmem<D>::kSubBytes + tensor * SparseSmem<D>::kTileBytes +
-                       tile_chunk_offset(r, c16),
-                   src, j >= 0 ? 16u : 0u);
+    constexpr int CH = D / 8;                       // 16-byte chunks per row
+    constexpr int RSTEP = kSparseThreads / CH;      // rows covered per pass
+    const int c16 = threadIdx.x % CH, r0 = threadIdx.x / CH;
+#pragma unroll
+    for (int sub = 0; sub < 2; ++sub) {
+#pragma unroll
+        for (int rr = r0; rr < kKeyTile; rr += RSTEP) {
+            const int j = s_idx[tile * kSparseTile + sub * kKeyTile + rr];
+            const int64_t off = (kv_base + (j >= 0 ? j : 0)) * D + c16 * 8;
+            const uint32_t nbytes = j >= 0 ? 16u : 0u;
+            uint8_t* dst = stage + sub * SparseSmem<D>::kSubBytes + tile_chunk_offset(rr, c16);
+            cp_async16(dst, a.K + off, nbytes);
+            cp_async16(dst + SparseSmem<D>::kTileBytes, a.V + off, nbytes);
+        }
     }
 }
 
