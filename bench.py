@@ -29,7 +29,7 @@ METRIC = "sparse-attn queries/s and achieved HBM GB/s (% of 8 TB/s) at N=128K, 1
 # DRAM bytes (read + write) per launch of the roofline kernel from an ncu capture of the same
 # kernel and workload (profiles/full_attn_long_decode.md); None where no capture matches the
 # current kernel.
-NCU_TRAFFIC = {("long", "full_attn_keep_logits"): 536923392 + 6701312}
+NCU_TRAFFIC = {("long", "full_attn_keep_logits"): 536923648 + 8172544}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
