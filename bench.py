@@ -26,9 +26,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn queries/s and achieved HBM GB/s (% of 8 TB/s) at N=128K, 1xB200"
-# DRAM bytes (read + write) per launch of the roofline kernel from an ncu capture of the same
-# kernel and workload (profiles/full_attn_long_decode.md); None where no capture matches the
-# current kernel.
+# DRAM bytes (read + write) per launch of the roofline kernel, from an ncu capture of the same
+# kernel binary on the same workload; None where no capture matches the current kernel.
 NCU_TRAFFIC = {("long", "full_attn_keep_logits"): 536923648 + 8172544}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
