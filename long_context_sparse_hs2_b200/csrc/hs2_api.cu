@@ -114,6 +114,11 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why) {
     P.cand_cap = P.fused ? x.N : std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
     const int64_t sparse_slots = std::max<int64_t>(P.S4, P.fused ? P.S1 : 0);
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
+    // multi-CTA top-k: one chunk per CTA while that is a few waves; with many chunks in all
+    // (1M keys x 64 rows) each CTA takes several, so launch and completion costs amortise
+    const int64_t nchunks = (static_cast<int64_t>(x.N) + kTopkChunk - 1) / kTopkChunk;
+    P.topk_ctas = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>(nchunks, std::max<int64_t>(1, (12 * int64_t(kSMs) + rows_kv - 1) / rows_kv))));
 
     size_t off = 0;
     P.off_status = off; off += 256;

@@ -51,6 +51,7 @@ struct Plan {
     int C4;             // selected keys per sparse-attention CTA
     int S4;             // sparse-attention splits per row = ceil((k+W)/C4)
     int64_t cand_cap;   // per-row capacity of the top-k candidate buffer
+    int topk_ctas;      // CTAs per row of the multi-CTA top-k kernels (each takes every topk_ctas-th chunk)
     int64_t kstride;    // row stride (elements) of the score-key buffer: N rounded up to 64
     bool fused;         // hs2_step runs the single fused decode-step kernel (T = 1, see k_decode.cu)
     // workspace byte offsets

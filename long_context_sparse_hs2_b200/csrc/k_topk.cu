@@ -33,18 +33,22 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(const TopkArgs a) {
     pdl_wait();  // keys from the score sweep (every CTA waits before it can finish)
     const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
     if (ri.keff == 0 || ri.keff == ri.P) return;
-    const int participants = (ri.P + kTopkChunk - 1) / kTopkChunk;
+    // the row's chunks are shared out over at most gridDim.x CTAs
+    const int nchunks = (ri.P + kTopkChunk - 1) / kTopkChunk;
+    const int participants = min(nchunks, static_cast<int>(gridDim.x));
     if (static_cast<int>(blockIdx.x) >= participants) return;
     __syncthreads();
-    const int j0 = blockIdx.x * kTopkChunk, j1 = min(j0 + kTopkChunk, ri.P);
     const uint32_t* keys = a.keys + row * a.kstride;
-    // 4 keys per thread per 16-byte load (rows are 256-byte aligned, j0 a multiple of 4)
-    for (int j = j0 + 4 * static_cast<int>(threadIdx.x); j < j1; j += 4 * blockDim.x) {
-        const uint4 q = __ldcs(reinterpret_cast<const uint4*>(keys + j));
-        const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
+    for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
+        const int j0 = c * kTopkChunk, j1 = min(j0 + kTopkChunk, ri.P);
+        // 4 keys per thread per 16-byte load (rows are 256-byte aligned, j0 a multiple of 4)
+        for (int j = j0 + 4 * static_cast<int>(threadIdx.x); j < j1; j += 4 * blockDim.x) {
+            const uint4 q = __ldcs(reinterpret_cast<const uint4*>(keys + j));
+            const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (j + e < j1) atomicAdd(&sh[score_bin(kk[e])], 1u);
+            for (int e = 0; e < 4; ++e)
+                if (j + e < j1) atomicAdd(&sh[score_bin(kk[e])], 1u);
+        }
     }
     __syncthreads();
     hist_flush_and_threshold(sh, a.hist + row * kHistBins, a.meta + row * kMetaInts, participants, ri.keff, s_warp,
@@ -192,7 +196,9 @@ __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
     static_assert(kTopkChunk % (4 * 256) == 0, "whole 16-byte key loads per thread");
     const int64_t row = blockIdx.y;
     const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
-    const int participants = max(1, (ri.P + kTopkChunk - 1) / kTopkChunk);
+    // the row's chunks are shared out over at most gridDim.x CTAs
+    const int nchunks = max(1, (ri.P + kTopkChunk - 1) / kTopkChunk);
+    const int participants = min(nchunks, static_cast<int>(gridDim.x));
     pdl_trigger();
     pdl_wait();  // keys, histogram threshold and cleared counters from the kernels before
     if (static_cast<int>(blockIdx.x) >= participants) return;
@@ -200,66 +206,70 @@ __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
     int32_t* idx = a.idx + row * kw;
     int32_t* out = idx + ri.wcnt;  // the pool's winners follow the window
     int* meta = a.meta + row * kMetaInts;
-    const int j0 = blockIdx.x * kTopkChunk, j1 = min(j0 + kTopkChunk, ri.P);
     const bool ranked = ri.keff > 0 && ri.keff < ri.P;
     const int b1 = ranked ? meta[kMetaBin] : 0;
     const int above = ranked ? meta[kMetaAbove] : 0;
 
-    if (ri.keff > 0 && ri.keff == ri.P) {  // the whole pool is selected
-        for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) out[j] = j;
-    } else if (ranked) {
-        const uint32_t* keys = a.keys + row * a.kstride;
-        unsigned long long* cand = a.cand + row * a.cand_cap;
-        // 16 keys per thread as four 16-byte loads; pass 1 counts, one global atomic per CTA
-        // reserves the CTA's slots, pass 2 writes with shared-memory slot counters.
-        constexpr int V4 = kTopkChunk / (4 * 256);
-        uint32_t kk[V4][4];
-        int bins[V4][4], ndef = 0, ncnd = 0;
-#pragma unroll
-        for (int v = 0; v < V4; ++v) {
-            const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v);
-            uint4 q = make_uint4(0, 0, 0, 0);
-            if (j < j1) q = __ldcs(reinterpret_cast<const uint4*>(keys + j));
-            kk[v][0] = q.x; kk[v][1] = q.y; kk[v][2] = q.z; kk[v][3] = q.w;
-        }
-#pragma unroll
-        for (int v = 0; v < V4; ++v)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v) + e;
-                bins[v][e] = j < j1 ? score_bin(kk[v][e]) : kHistBins;
-                ndef += bins[v][e] < b1;
-                ncnd += bins[v][e] == b1;
+    for (int chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
+        const int j0 = chunk * kTopkChunk, j1 = min(j0 + kTopkChunk, ri.P);
+        if (ri.keff > 0 && ri.keff == ri.P) {  // the whole pool is selected
+            for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) out[j] = j;
+        } else if (ranked) {
+            const uint32_t* keys = a.keys + row * a.kstride;
+            unsigned long long* cand = a.cand + row * a.cand_cap;
+            // 16 keys per thread as four 16-byte loads; pass 1 counts, one global atomic per CTA
+            // reserves the CTA's slots, pass 2 writes with shared-memory slot counters.
+            constexpr int V4 = kTopkChunk / (4 * 256);
+            uint32_t kk[V4][4];
+            int bins[V4][4], ndef = 0, ncnd = 0;
+    #pragma unroll
+            for (int v = 0; v < V4; ++v) {
+                const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v);
+                uint4 q = make_uint4(0, 0, 0, 0);
+                if (j < j1) q = __ldcs(reinterpret_cast<const uint4*>(keys + j));
+                kk[v][0] = q.x; kk[v][1] = q.y; kk[v][2] = q.z; kk[v][3] = q.w;
             }
-        if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
-        __syncthreads();
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
-            ncnd += __shfl_xor_sync(0xffffffffu, ncnd, o);
-        }
-        if ((threadIdx.x & 31) == 0) {
-            atomicAdd(&s_cnt[0], ndef);
-            atomicAdd(&s_cnt[1], ncnd);
-        }
-        __syncthreads();
-        const int2 bases = block_reserve2(s_cnt[0], s_cnt[1], &meta[kMetaDef], &s_base2);
-        const int def_base = bases.x, cnd_base = bases.y;
-        if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
-        __syncthreads();
-#pragma unroll
-        for (int v = 0; v < V4; ++v)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v) + e;
-                const bool def = bins[v][e] < b1;
-                const bool cnd = bins[v][e] == b1;
-                const int sd = warp_append(def, &s_cnt[0]);
-                if (def && def_base + sd < above) out[def_base + sd] = j;
-                const int sc = warp_append(cnd, &s_cnt[1]);
-                if (cnd && cnd_base + sc < a.cand_cap) cand[cnd_base + sc] = composite(kk[v][e], j);
+    #pragma unroll
+            for (int v = 0; v < V4; ++v)
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v) + e;
+                    bins[v][e] = j < j1 ? score_bin(kk[v][e]) : kHistBins;
+                    ndef += bins[v][e] < b1;
+                    ncnd += bins[v][e] == b1;
+                }
+            if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
+            __syncthreads();
+    #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                ndef += __shfl_xor_sync(0xffffffffu, ndef, o);
+                ncnd += __shfl_xor_sync(0xffffffffu, ncnd, o);
             }
-    }
+            if ((threadIdx.x & 31) == 0) {
+                atomicAdd(&s_cnt[0], ndef);
+                atomicAdd(&s_cnt[1], ncnd);
+            }
+            __syncthreads();
+            const int2 bases = block_reserve2(s_cnt[0], s_cnt[1], &meta[kMetaDef], &s_base2);
+            const int def_base = bases.x, cnd_base = bases.y;
+            if (threadIdx.x == 0) s_cnt[0] = s_cnt[1] = 0;
+            __syncthreads();
+    #pragma unroll
+            for (int v = 0; v < V4; ++v)
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j0 + 4 * (static_cast<int>(threadIdx.x) + 256 * v) + e;
+                    const bool def = bins[v][e] < b1;
+                    const bool cnd = bins[v][e] == b1;
+                    const int sd = warp_append(def, &s_cnt[0]);
+                    if (def && def_base + sd < above) out[def_base + sd] = j;
+                    const int sc = warp_append(cnd, &s_cnt[1]);
+                    if (cnd && cnd_base + sc < a.cand_cap) cand[cnd_base + sc] = composite(kk[v][e], j);
+                }
+            __syncthreads();  // the slot counters are reset for the next chunk
+        }
+
+    }  // chunks
 
     // completion: the row's last CTA finishes the row
     __threadfence();
@@ -534,14 +544,14 @@ cudaError_t launch_topk_rows(const Plan& p, const TopkArgs& a, cudaStream_t st) 
 }
 
 cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st) {
-    dim3 grid((p.N + kTopkChunk - 1) / kTopkChunk, static_cast<unsigned>(p.rows_kv));
+    dim3 grid(p.topk_ctas, static_cast<unsigned>(p.rows_kv));
     const cudaError_t e = launch_pdl(topk_hist_kernel, grid, dim3(256), 0, st, a);
     trace_mark("topk_hist", st);
     return e;
 }
 
 cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st) {
-    dim3 grid((p.N + kTopkChunk - 1) / kTopkChunk, static_cast<unsigned>(p.rows_kv));
+    dim3 grid(p.topk_ctas, static_cast<unsigned>(p.rows_kv));
     const cudaError_t e = launch_pdl(topk_select_kernel, grid, dim3(256), 0, st, a);
     trace_mark("topk_select", st);
     return e;

@@ -160,3 +160,20 @@ def test_many_rows_large_pools_all_ties_fall_back():
     ref = compare_step(inp, res, rows=rows)
     for (b, h, t), r in ref.items():
         np.testing.assert_array_equal(np.sort(res["idx"][b, h, t][:res["cnt"][b, h, t]]), r.selected)
+
+
+def test_multi_cta_topk_with_several_chunks_per_cta():
+    # 400 selection rows of ~40 K keys: the multi-CTA top-k gives each CTA several 4096-key
+    # chunks (fewer CTAs than chunks per row); sampled rows against the oracle, every row's
+    # invariants
+    from tests.test_gpu_parity import compare_step, run_step
+    from tests.test_gpu_workloads import check_all_rows
+
+    inp = make_inputs(1, 8, 1, 128, 40000, 400, 2048, 128, seed=25, needles=32)
+    hs2.trace_enable(True)
+    res = run_step(inp)
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    assert "topk_select" in kernels and "topk_rows" not in kernels, kernels
+    check_all_rows(inp, res["idx"], res["cnt"])
+    compare_step(inp, res, rows=[(0, 0, t) for t in (0, 133, 200, 399)])
