@@ -393,8 +393,8 @@ def main():
     cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "T": w.T, "k": w.k,
            "W": w.W, "global_batch": w.B * w.T * max(world, args.gpus), "seq_len": w.N,
            "parallelism": f"replicas x{max(world, args.gpus)}",
-           "l2": (("flush: a %d MiB buffer is written between timed steps (K and V, %d MiB, fit in the 126 MB L2)"
-                   % (L2_FLUSH_BYTES >> 20, kv_bytes(w) >> 20)) if kv_fits_l2(w) else
+           "l2": (("flush: a %d MiB buffer is written between timed steps (K and V, %.1f MiB, fit in the 126 MB L2)"
+                   % (L2_FLUSH_BYTES >> 20, kv_bytes(w) / 2**20)) if kv_fits_l2(w) else
                   "no flush: K and V (%d MiB) exceed the 126 MB L2" % (kv_bytes(w) >> 20))}
 
     if args.impl == "reference":
