@@ -56,6 +56,24 @@ def test_workspace_size(L):
     assert L.hs2_workspace_size(None) == 0
 
 
+def test_workspace_follows_the_execution_plan(L, monkeypatch):
+    # 128-row query tiles (T*G > 64) run on the tcgen05 sweeps unless HS2_UMMA=0; the split
+    # partials, and so the workspace, depend on the plan.  Every supported shape has a size.
+    prefill = _dims(Hq=32, Hkv=4, T=4096, N=131072, k=2048, W=128)
+    t16 = _dims(Hq=32, Hkv=4, T=16, N=1 << 20, k=8192, W=1024)
+    sizes = {}
+    for umma in ("1", "0"):
+        monkeypatch.setenv("HS2_UMMA", umma)
+        sizes[umma] = (hs2.workspace_size(prefill), hs2.workspace_size(t16))
+        assert all(v > 0 and v % 256 == 0 for v in sizes[umma])
+    assert sizes["1"] != sizes["0"]
+    monkeypatch.delenv("HS2_UMMA")
+    assert (hs2.workspace_size(prefill), hs2.workspace_size(t16)) == sizes["1"]  # the default is tcgen05
+    for G in (1, 2, 4, 8, 16):
+        for d in (64, 128):
+            assert hs2.workspace_size(_dims(Hq=G, Hkv=1, T=max(1, 200 // G), N=5000, d=d)) > 0, (G, d)
+
+
 FAKE = 1 << 20  # a 256-byte-aligned non-null address; never dereferenced (checks fail first)
 
 
