@@ -13,7 +13,7 @@
 //               CTA's key range (few query tiles, e.g. 16 decode queries), and each stream
 //               writes its own split partial.
 //
-// Roles (320 threads):
+// Roles (384 threads):
 //   warps 0-3   softmax of stream 0 (thread = TMEM lane = tile row), warps 4-7 stream 1
 //   warp 8      TMA producer: K and V tiles of 128 keys into two 2-stage rings
 //   warp 9      allocates TMEM; one lane issues every tcgen05.mma and commit
@@ -25,8 +25,10 @@
 // Per stream and key tile: S = Q K^T (SS MMA, K-major operands) -> softmax warps read S,
 // mask, update the running max with lazy rescaling (O and l are rescaled only when the max
 // grows by more than 8 in base-2 units, exact because the final normalisation uses the same
-// reference max), write P = 2^(S - m) into TMEM -> O += P V (TS MMA, V MN-major).  Every
-// wait is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains and exits.
+// reference max), write P = 2^(S - m) into TMEM -> O += P V (TS MMA, V MN-major).  The row
+// max uses three-input maxes in independent chains, the scaling and the row sum run on packed
+// f32x2 pairs.  Every wait is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains and
+// exits.
 //
 // The split partials (m, l, O) and the log-sum-exp combine are those of the mma.sync sweep
 // ("Simplified Sparse Attention via Gist Tokens", section 3.6, split-K flash-decode).
