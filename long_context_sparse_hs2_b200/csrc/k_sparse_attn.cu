@@ -11,10 +11,10 @@
 //
 // Grid: (S4 splits, B*Hkv*T rows).  A CTA reads its C4 slots of the row's index list,
 // validates them (0 <= j <= pos; others are skipped and flagged), gathers the rows with
-// 16-byte cp.async into the same 128-byte-swizzled tile layout the TMA path uses -- up to
-// four 64-key tiles in flight -- and runs the shared warp attention core.  The row's last
-// CTA to finish (a completion counter; nothing waits) merges the S4 split partials into
-// O_sparse and LSE_sparse.
+// 16-byte cp.async into the same 128-byte-swizzled tile layout the TMA path uses -- a ring
+// of up to three 128-key steps in flight -- and runs the shared warp attention core.  The
+// row's last CTA to finish (a completion counter; nothing waits) merges the S4 split
+// partials into O_sparse and LSE_sparse.
 #include <algorithm>
 
 #include "attn_core.cuh"

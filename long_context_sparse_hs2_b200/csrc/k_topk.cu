@@ -9,7 +9,8 @@
 //
 // The scores arrive as order-preserving keys with a per-row histogram of a monotone
 // bucketing and the threshold bucket b1 already found (score_hist_kernel, or
-// topk_hist_kernel below after a K re-sweep).  topk_select_kernel then:
+// topk_hist_kernel below after a K re-sweep); each CTA takes every gridDim.x-th 4096-key
+// chunk of its row.  topk_select_kernel then:
 //   * selects every key in a better bucket than b1 outright and appends the keys of b1 to a
 //     candidate list (warp ballot + one atomic per warp; order arbitrary -- the compaction
 //     pattern of "Simplified Sparse Attention via Gist Tokens", section 3.6);
@@ -17,6 +18,7 @@
 //     the exact 64-bit composite threshold among the candidates, emits the winners, and
 //     writes the window, the -1 padding and cnt.  If the candidate list overflowed its
 //     capacity it re-scans the row's keys instead (exact, slower, flagged).
+// With thousands of rows topk_rows_kernel (further below) finishes each row in one CTA.
 #include "topk_common.cuh"
 
 namespace hs2 {
