@@ -79,10 +79,7 @@ __device__ __forceinline__ int2 block_reserve2(int n0, int n1, int* ctr, unsigne
     if (threadIdx.x == 0) {
         const unsigned long long add = (static_cast<unsigned long long>(static_cast<unsigned>(n1)) << 32) |
                                        static_cast<unsigned>(n0);
-        *s_base = add ? atomicAdd(reinterpret_cast<unsigned long long*>(ctr), add) : 0ull;
-        if (!add) {
-            // nothing to reserve: the bases are not needed
-        }
+        *s_base = add ? atomicAdd(reinterpret_cast<unsigned long long*>(ctr), add) : 0ull;  // nothing to reserve: unused
     }
     __syncthreads();
     const unsigned long long v = *s_base;
