@@ -158,7 +158,9 @@ HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void
  *    are rejected with HS2_ERR_WORKSPACE before anything is launched; decode shapes up to a
  *    few hundred query-head rows fit.
  *  - Set-up: the first call on each device looks up the array's device address (while that
- *    device is current); make that first call before any stream capture.
+ *    device is current); make that first call before any stream capture.  The address is kept
+ *    for the life of the process: do not call this entry point after cudaDeviceReset, which
+ *    frees the array and leaves the kept address dangling.
  *  - Sharing: every call on a device uses the same array and leaves its contents behind; each
  *    call clears what must start at zero.  Calls whose GPU work overlaps (other streams, other
  *    host threads) race on the array and give undefined results: serialise them.

@@ -12,7 +12,8 @@
 // The kernels are the ones hs2_sparse_attn launches; only where their scratch lives differs.
 // Host code cannot use the array's name as a device address (it stands for a host-side shadow),
 // so the first call on each device looks the address up with cudaGetSymbolAddress while that
-// device is current, and later calls reuse it.
+// device is current, and later calls reuse it.  The cached address belongs to the device context
+// it was looked up in: after cudaDeviceReset the array is reallocated and the cache is stale.
 #include <mutex>
 
 #include "hs2_internal.h"
@@ -77,6 +78,7 @@ extern "C" hs2_status hs2_sparse_attn_static(const hs2_dims* dims, const void* Q
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     // the array keeps the previous call's contents: clear the status word and the counters
+    trace_call_begin(st);
     if (launch_init(base, meta_end, st) != cudaSuccess) return HS2_ERR_CUDA;
     SparseArgs sa{};
     sa.Q = static_cast<const uint16_t*>(Q_sparse);

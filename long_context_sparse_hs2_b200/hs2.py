@@ -106,10 +106,29 @@ def _p(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream) -> Optional[int]:
+def _stream(stream, device) -> Optional[int]:
+    """Raw handle of ``stream`` (default: the current stream of ``device``).  A torch stream must
+    belong to ``device``: the library launches on whatever device is current, so a stream of
+    another GPU would run the kernels there."""
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        stream = torch.cuda.current_stream(device)
+    if hasattr(stream, "cuda_stream"):
+        if getattr(stream, "device", device) != device:
+            raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
+        return stream.cuda_stream
+    return int(stream)
+
+
+def device_of(where: str, **tensors) -> torch.device:
+    """The one CUDA device every given tensor lives on (``None`` entries are skipped).
+
+    The kernels run on the current device and dereference every pointer there, so tensors on
+    two GPUs would read the wrong memory or fault: this raises before anything is launched."""
+    devs = {name: t.device for name, t in tensors.items() if t is not None}
+    if len(set(devs.values())) != 1:
+        listing = ", ".join(f"{n} on {d}" for n, d in devs.items())
+        raise ValueError(f"{where}: every tensor must be on one CUDA device ({listing})")
+    return next(iter(devs.values()))
 
 
 def _need(t: torch.Tensor, name: str, dtype, shape):
@@ -150,11 +169,13 @@ def full_attn(Q_full, K, V, pos, *, k: int = 0, W: int = 0, O_full=None, LSE_ful
     _need(K, "K", torch.bfloat16, (B, Hkv, N, d))
     _need(V, "V", torch.bfloat16, (B, Hkv, N, d))
     _need(pos, "pos", torch.int32, (B, T))
-    O_full = torch.empty_like(Q_full) if O_full is None else O_full
-    LSE_full = torch.empty((B, Hq, T), dtype=torch.float32, device=Q_full.device) if LSE_full is None else LSE_full
-    ws = _ws(dm, ws, Q_full.device)
-    _check(lib().hs2_full_attn(ctypes.byref(dm), _p(Q_full), _p(K), _p(V), _p(pos), _p(O_full), _p(LSE_full),
-                               _p(ws), ws.numel(), _stream(stream)), "hs2_full_attn")
+    dev = device_of("full_attn", Q_full=Q_full, K=K, V=V, pos=pos, O_full=O_full, LSE_full=LSE_full, ws=ws)
+    with torch.cuda.device(dev):
+        O_full = torch.empty_like(Q_full) if O_full is None else O_full
+        LSE_full = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if LSE_full is None else LSE_full
+        ws = _ws(dm, ws, dev)
+        _check(lib().hs2_full_attn(ctypes.byref(dm), _p(Q_full), _p(K), _p(V), _p(pos), _p(O_full), _p(LSE_full),
+                                   _p(ws), ws.numel(), _stream(stream, dev)), "hs2_full_attn")
     return O_full, LSE_full
 
 
@@ -166,17 +187,17 @@ def select(Q_full, K, LSE_full, pos, *, k: int, W: int, idx=None, cnt=None, ws=N
     _need(K, "K", torch.bfloat16, (B, Hkv, N, d))
     _need(LSE_full, "LSE_full", torch.float32, (B, Hq, T))
     _need(pos, "pos", torch.int32, (B, T))
-    idx = torch.empty((B, Hkv, T, k + W), dtype=torch.int32, device=K.device) if idx is None else idx
-    cnt = torch.empty((B, Hkv, T), dtype=torch.int32, device=K.device) if cnt is None else cnt
-    ws = _ws(dm, ws, K.device)
-    _check(lib().hs2_select(ctypes.byref(dm), _p(Q_full), _p(K), _p(LSE_full), _p(pos), _p(idx), _p(cnt),
-                            _p(ws), ws.numel(), _stream(stream)), "hs2_select")
+    dev = device_of("select", Q_full=Q_full, K=K, LSE_full=LSE_full, pos=pos, idx=idx, cnt=cnt, ws=ws)
+    with torch.cuda.device(dev):
+        idx = torch.empty((B, Hkv, T, k + W), dtype=torch.int32, device=dev) if idx is None else idx
+        cnt = torch.empty((B, Hkv, T), dtype=torch.int32, device=dev) if cnt is None else cnt
+        ws = _ws(dm, ws, dev)
+        _check(lib().hs2_select(ctypes.byref(dm), _p(Q_full), _p(K), _p(LSE_full), _p(pos), _p(idx), _p(cnt),
+                                _p(ws), ws.numel(), _stream(stream, dev)), "hs2_select")
     return idx, cnt
 
 
-def sparse_attn(Q_sparse, K, V, pos, idx, cnt, *, k: int, W: int, O_sparse=None, LSE_sparse=None, ws=None,
-                stream=None):
-    """Sparse layer with KV Reuse over idx/cnt: returns (O_sparse bf16, LSE_sparse fp32)."""
+def _sparse_checks(where, Q_sparse, K, V, pos, idx, cnt, k, W, O_sparse, LSE_sparse, ws=None):
     dm = dims_of(Q_sparse, K, k, W)
     B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
     _need(Q_sparse, "Q_sparse", torch.bfloat16, (B, Hq, T, d))
@@ -185,12 +206,23 @@ def sparse_attn(Q_sparse, K, V, pos, idx, cnt, *, k: int, W: int, O_sparse=None,
     _need(pos, "pos", torch.int32, (B, T))
     _need(idx, "idx", torch.int32, (B, Hkv, T, k + W))
     _need(cnt, "cnt", torch.int32, (B, Hkv, T))
-    O_sparse = torch.empty_like(Q_sparse) if O_sparse is None else O_sparse
-    LSE_sparse = torch.empty((B, Hq, T), dtype=torch.float32, device=K.device) if LSE_sparse is None else LSE_sparse
-    ws = _ws(dm, ws, K.device)
-    _check(lib().hs2_sparse_attn(ctypes.byref(dm), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(idx), _p(cnt),
-                                 _p(O_sparse), _p(LSE_sparse), _p(ws), ws.numel(), _stream(stream)),
-           "hs2_sparse_attn")
+    dev = device_of(where, Q_sparse=Q_sparse, K=K, V=V, pos=pos, idx=idx, cnt=cnt, O_sparse=O_sparse,
+                    LSE_sparse=LSE_sparse, ws=ws)
+    return dm, dev
+
+
+def sparse_attn(Q_sparse, K, V, pos, idx, cnt, *, k: int, W: int, O_sparse=None, LSE_sparse=None, ws=None,
+                stream=None):
+    """Sparse layer with KV Reuse over idx/cnt: returns (O_sparse bf16, LSE_sparse fp32)."""
+    dm, dev = _sparse_checks("sparse_attn", Q_sparse, K, V, pos, idx, cnt, k, W, O_sparse, LSE_sparse, ws)
+    B, Hq, _, T = dm.B, dm.Hq, dm.Hkv, dm.T
+    with torch.cuda.device(dev):
+        O_sparse = torch.empty_like(Q_sparse) if O_sparse is None else O_sparse
+        LSE_sparse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if LSE_sparse is None else LSE_sparse
+        ws = _ws(dm, ws, dev)
+        _check(lib().hs2_sparse_attn(ctypes.byref(dm), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(idx), _p(cnt),
+                                     _p(O_sparse), _p(LSE_sparse), _p(ws), ws.numel(), _stream(stream, dev)),
+               "hs2_sparse_attn")
     return O_sparse, LSE_sparse
 
 
@@ -198,18 +230,14 @@ def sparse_attn_static(Q_sparse, K, V, pos, idx, cnt, *, k: int, W: int, O_spars
                        stream=None):
     """hs2_sparse_attn_static: the sparse layer with its scratch in the library's fixed device
     array (no workspace).  The outputs are allocated here only if the caller passes none."""
-    dm = dims_of(Q_sparse, K, k, W)
-    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
-    _need(Q_sparse, "Q_sparse", torch.bfloat16, (B, Hq, T, d))
-    _need(K, "K", torch.bfloat16, (B, Hkv, N, d))
-    _need(V, "V", torch.bfloat16, (B, Hkv, N, d))
-    _need(pos, "pos", torch.int32, (B, T))
-    _need(idx, "idx", torch.int32, (B, Hkv, T, k + W))
-    _need(cnt, "cnt", torch.int32, (B, Hkv, T))
-    O_sparse = torch.empty_like(Q_sparse) if O_sparse is None else O_sparse
-    LSE_sparse = torch.empty((B, Hq, T), dtype=torch.float32, device=K.device) if LSE_sparse is None else LSE_sparse
-    _check(lib().hs2_sparse_attn_static(ctypes.byref(dm), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(idx), _p(cnt),
-                                        _p(O_sparse), _p(LSE_sparse), _stream(stream)), "hs2_sparse_attn_static")
+    dm, dev = _sparse_checks("sparse_attn_static", Q_sparse, K, V, pos, idx, cnt, k, W, O_sparse, LSE_sparse)
+    B, Hq, T = dm.B, dm.Hq, dm.T
+    with torch.cuda.device(dev):
+        O_sparse = torch.empty_like(Q_sparse) if O_sparse is None else O_sparse
+        LSE_sparse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if LSE_sparse is None else LSE_sparse
+        _check(lib().hs2_sparse_attn_static(ctypes.byref(dm), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(idx),
+                                            _p(cnt), _p(O_sparse), _p(LSE_sparse), _stream(stream, dev)),
+               "hs2_sparse_attn_static")
     return O_sparse, LSE_sparse
 
 
@@ -248,18 +276,22 @@ def step(Q_full, Q_sparse, K, V, pos, *, k: int, W: int, out: Optional[StepOutpu
     _need(K, "K", torch.bfloat16, (B, Hkv, N, d))
     _need(V, "V", torch.bfloat16, (B, Hkv, N, d))
     _need(pos, "pos", torch.int32, (B, T))
-    out = alloc_step_outputs(dm, K.device) if out is None else out
-    ws = _ws(dm, ws, K.device)
-    _check(lib().hs2_step(ctypes.byref(dm), _p(Q_full), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(out.O_full),
-                          _p(out.O_sparse), _p(out.LSE_full), _p(out.LSE_sparse), _p(out.idx), _p(out.cnt),
-                          _p(ws), ws.numel(), _stream(stream)), "hs2_step")
+    outs = out.as_dict() if out is not None else {}
+    dev = device_of("step", Q_full=Q_full, Q_sparse=Q_sparse, K=K, V=V, pos=pos, ws=ws, **outs)
+    with torch.cuda.device(dev):
+        out = alloc_step_outputs(dm, dev) if out is None else out
+        ws = _ws(dm, ws, dev)
+        _check(lib().hs2_step(ctypes.byref(dm), _p(Q_full), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(out.O_full),
+                              _p(out.O_sparse), _p(out.LSE_full), _p(out.LSE_sparse), _p(out.idx), _p(out.cnt),
+                              _p(ws), ws.numel(), _stream(stream, dev)), "hs2_step")
     return out
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:
     """Device status bits of the last call that used ``ws`` (synchronises the stream)."""
     bits = ctypes.c_uint32(0)
-    st = lib().hs2_read_device_status(_p(ws), _stream(stream), ctypes.byref(bits))
+    with torch.cuda.device(ws.device):
+        st = lib().hs2_read_device_status(_p(ws), _stream(stream, ws.device), ctypes.byref(bits))
     if st not in (HS2_OK, HS2_ERR_DEVICE):
         raise HS2Error(st, "hs2_read_device_status")
     return int(bits.value)

@@ -132,3 +132,18 @@ def test_selection_checker_accepts_oracle_and_rejects_wrong_sets():
         row[:len(bad)] = bad
         with pytest.raises(AssertionError):
             parity.check_selection(row, cnt, r)
+
+
+def test_python_binding_refuses_tensors_on_two_devices():
+    # the library launches on the current device and dereferences every pointer there, so the
+    # binding must refuse a call whose tensors sit on two GPUs before anything is launched
+    import types
+
+    import torch
+
+    on = lambda i: types.SimpleNamespace(device=torch.device("cuda", i))  # noqa: E731
+    assert hs2.device_of("t", Q=on(1), K=on(1), ws=None) == torch.device("cuda", 1)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        hs2.device_of("t", Q=on(0), K=on(1))
+    with pytest.raises(ValueError, match="one CUDA device"):
+        hs2.device_of("t", Q=on(0), K=on(0), ws=on(1))
