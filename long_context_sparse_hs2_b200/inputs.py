@@ -105,8 +105,41 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------- inputs
 
 @dataclass
+class KVCache:
+    """The shared KV cache as it is stored, when it is not plain contiguous bf16.
+
+    dtype "bf16": K/V hold bfloat16 bit patterns (uint16).  dtype "fp8_e4m3": K/V hold FP8
+    E4M3 codes (uint8) and a token's value is code * scale, with one fp32 scale per
+    (b, kv head) for K and one for V.  Contiguous layout: K/V are [B, Hkv, N, d].  Paged
+    layout (page_size > 0): K/V are a pool [num_pages, Hkv, page_size, d] and token j of
+    batch row b sits in page page_table[b, j // page_size] at slot j % page_size.
+    """
+
+    dtype: str
+    K: np.ndarray
+    V: np.ndarray
+    N: int
+    k_scale: Optional[np.ndarray] = None    # float32 [B, Hkv] (fp8 only)
+    v_scale: Optional[np.ndarray] = None
+    page_size: int = 0
+    page_table: Optional[np.ndarray] = None  # int32 [B, max_pages] (paged only)
+
+    @property
+    def Hkv(self) -> int:
+        return self.K.shape[1]
+
+    def copy(self) -> "KVCache":
+        c = lambda a: None if a is None else a.copy()  # noqa: E731
+        return replace(self, K=self.K.copy(), V=self.V.copy(), k_scale=c(self.k_scale), v_scale=c(self.v_scale),
+                       page_table=c(self.page_table))
+
+
+@dataclass
 class Inputs:
-    """One step's inputs as bf16 bit patterns plus the integer arguments."""
+    """One step's inputs as bf16 bit patterns plus the integer arguments.
+
+    ``cache`` replaces K/V when the cache is stored in another format or layout (then K and V
+    keep the bf16 draw it was made from, for reference only)."""
 
     Qf: np.ndarray          # uint16 [B, Hq, T, d]
     Qs: np.ndarray          # uint16 [B, Hq, T, d]
@@ -116,11 +149,15 @@ class Inputs:
     k: int
     W: int
     needle_pos: np.ndarray = field(default_factory=lambda: np.zeros((0,), np.int64))
+    cache: Optional[KVCache] = None
 
     @property
     def dims(self):
         B, Hq, T, d = self.Qf.shape
-        Hkv, N = self.K.shape[1], self.K.shape[2]
+        if self.cache is not None:
+            Hkv, N = self.cache.Hkv, self.cache.N
+        else:
+            Hkv, N = self.K.shape[1], self.K.shape[2]
         return dict(B=B, Hq=Hq, Hkv=Hkv, T=T, N=N, d=d, k=self.k, W=self.W)
 
 
@@ -192,3 +229,106 @@ def generate(w: Workload, **overrides) -> Inputs:
         w = replace(w, **overrides)
     return make_inputs(w.B, w.Hq, w.Hkv, w.d, w.N, w.T, w.k, w.W, w.seed,
                        needles=w.needles, drift=w.drift)
+
+
+# ----------------------------------------------------------------------------- cache formats
+
+FP8_E4M3_MAX = 448.0
+
+
+def fp8_e4m3_cache(K_bits: np.ndarray, V_bits: np.ndarray) -> KVCache:
+    """FP8 E4M3 image of a bf16 cache [B, Hkv, N, d] with one amax scale per (b, kv head).
+
+    scale = max|x| / 448 in float32, code = the float32 quotient x / scale rounded to E4M3
+    (nearest, ties to even; PyTorch's float8_e4m3fn conversion).  This is how the synthetic
+    fp8 workloads are stored; it is data preparation, done once per workload."""
+    import torch
+
+    B, Hkv = K_bits.shape[:2]
+    out = []
+    for bits in (K_bits, V_bits):
+        codes = np.empty(bits.shape, np.uint8)
+        scale = np.empty((B, Hkv), np.float32)
+        for b in range(B):
+            for h in range(Hkv):
+                x = bf16_bits_to_f32(bits[b, h])
+                amax = np.float32(np.abs(x).max())
+                sc = np.float32(amax / np.float32(FP8_E4M3_MAX)) if amax > 0 else np.float32(1.0)
+                q = np.clip(x / sc, -FP8_E4M3_MAX, FP8_E4M3_MAX).astype(np.float32)
+                codes[b, h] = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+                scale[b, h] = sc
+        out.append((codes, scale))
+    (K8, ks), (V8, vs) = out
+    return KVCache("fp8_e4m3", K8, V8, N=K_bits.shape[2], k_scale=ks, v_scale=vs)
+
+
+def bf16_cache(inp: Inputs) -> KVCache:
+    """The inputs' own contiguous bf16 cache as a KVCache."""
+    return KVCache("bf16", inp.K, inp.V, N=inp.K.shape[2])
+
+
+def paged_cache(c: KVCache, page_size: int, seed: int, spare_pages: int = 3) -> KVCache:
+    """The same cache in a paged pool [num_pages, Hkv, page_size, d] with a shuffled page table.
+
+    Every batch row owns ceil(N / page_size) pages; the pool also holds ``spare_pages`` pages no
+    row uses, and the physical order of all pages is a seeded random permutation.  Slots past N
+    in a row's last page and the spare pages are filled with junk (all bytes 0x7F: NaN in both
+    bf16 and E4M3), so a read of anything but the mapped tokens shows in the results."""
+    if c.page_size:
+        raise ValueError("already paged")
+    B, Hkv, N, d = c.K.shape
+    per = -(-N // page_size)
+    num = B * per + spare_pages
+    rng = np.random.Generator(np.random.PCG64(seed))
+    perm = rng.permutation(num).astype(np.int32)
+    table = perm[:B * per].reshape(B, per).copy()
+    pools = []
+    for x in (c.K, c.V):
+        pool = np.full((num, Hkv, page_size, d), 0x7F, dtype=x.dtype)
+        if x.dtype == np.uint16:
+            pool[...] = 0x7F7F
+        for b in range(B):
+            for i in range(per):
+                j0, j1 = i * page_size, min(N, (i + 1) * page_size)
+                pool[table[b, i], :, :j1 - j0] = x[b, :, j0:j1]
+        pools.append(pool)
+    return replace(c, K=pools[0], V=pools[1], page_size=page_size, page_table=table)
+
+
+@dataclass
+class DecodeSteps:
+    """Inputs of a run of consecutive decode steps: each step appends one token per batch row
+    to the cache and then runs the hybrid step for that token as the query (T = 1).
+
+    ``start`` is the cache before the first step (``start.pos[b, 0]`` = the newest token already
+    cached); step s brings Q_full/Q_sparse [B, Hq, 1, d] and the new token's K/V [B, Hkv, d]."""
+
+    start: Inputs
+    Qf: np.ndarray      # uint16 [S, B, Hq, 1, d]
+    Qs: np.ndarray      # uint16 [S, B, Hq, 1, d]
+    K_new: np.ndarray   # uint16 [S, B, Hkv, d]
+    V_new: np.ndarray   # uint16 [S, B, Hkv, d]
+
+
+def make_decode_steps(start: Inputs, steps: int, seed: int, drift: float = 0.0) -> DecodeSteps:
+    """Draw ``steps`` decode steps after ``start``: new tokens' K/V ~ N(0,1); each query is the
+    previous query plus ``drift``-scaled N(0,1) noise (0: independent N(0,1) queries), the
+    first one continuing from the start's last query."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    B, Hq, T, d = start.Qf.shape
+    Hkv = start.dims["Hkv"]
+    qf, qs = bf16_bits_to_f32(start.Qf[:, :, -1:]), bf16_bits_to_f32(start.Qs[:, :, -1:])
+    Qf, Qs = [], []
+    for _ in range(steps):
+        nf = rng.standard_normal(qf.shape, dtype=np.float32)
+        ns = rng.standard_normal(qs.shape, dtype=np.float32)
+        if drift > 0:
+            qf = (qf + np.float32(drift) * nf) / np.float32(np.sqrt(1 + drift * drift))
+            qs = (qs + np.float32(drift) * ns) / np.float32(np.sqrt(1 + drift * drift))
+        else:
+            qf, qs = nf, ns
+        Qf.append(f32_to_bf16_bits(qf))
+        Qs.append(f32_to_bf16_bits(qs))
+    K_new = f32_to_bf16_bits(rng.standard_normal((steps, B, Hkv, d), dtype=np.float32))
+    V_new = f32_to_bf16_bits(rng.standard_normal((steps, B, Hkv, d), dtype=np.float32))
+    return DecodeSteps(start=start, Qf=np.stack(Qf), Qs=np.stack(Qs), K_new=K_new, V_new=V_new)

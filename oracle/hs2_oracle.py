@@ -36,11 +36,26 @@ the top-k pool open.  This library fixes them, and the oracle follows:
 4. sparse attention (KV Reuse): the full-attention definition with Q_sparse,
    restricted to the selected keys, the same index set for all G query heads of
    kv head h.
+
+The shared cache may be stored in other ways than contiguous bf16 (the pages
+give no storage format; the 2.69 GB cache figure comes without its precision:
+"HySparse2 od Xiaomi zkracuje zpracování dlouhého kontextu", section "Co říkají
+výsledky — a co z nich neplyne").  The oracle reads every stored form back to
+exact float64 values first (section "KV cache as stored" below) and then applies
+the same four definitions:
+
+* FP8 E4M3 codes with one fp32 scale per (b, kv head) for K and one for V: the
+  value of a code is its exact E4M3 value times the scale;
+* a paged pool: token j of batch row b lives in page page_table[b][j // page_size]
+  at slot j % page_size;
+* a run of decode steps: each step first writes the new token's K/V at position
+  pos + 1 (rounded to E4M3 for an fp8 cache) and then computes the step for a
+  query at that position.
 """
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 from typing import Dict, Iterable, List, Optional, Tuple
 
 import numpy as np
@@ -86,6 +101,105 @@ def attend(q: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, scale: float):
     lse = m[:, 0] + np.log(np.exp(logits - m).sum(axis=1))
     p = np.exp(logits - lse[:, None])
     return p @ Vh, lse, logits
+
+
+# ----------------------------------------------------------------------------- KV cache as stored
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Exact value of FP8 E4M3 codes: sign bit, 4 exponent bits (bias 7), 3 mantissa bits.
+
+    Exponent field 0 is subnormal, (m / 8) * 2^-6; otherwise (1 + m / 8) * 2^(e - 7).  The
+    codes S.1111.111 are NaN; the format has no infinities (largest finite value 448)."""
+    c = np.asarray(codes).astype(np.int64)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return np.where(c & 0x80, -mag, mag)
+
+
+def quantize_e4m3(x_f32: np.ndarray, scale: float) -> np.ndarray:
+    """E4M3 code of the float32 quotient x / scale: round to nearest, ties to even, magnitudes
+    beyond 448 saturate to 448 (codes 0x7E / 0xFE), NaN gives 0x7F.
+
+    The quotient is one IEEE float32 division (the precision the rounding decision is taken
+    in); the rounding itself is done exactly in float64 on that quotient."""
+    v = (np.asarray(x_f32, np.float32) / np.float32(scale)).astype(np.float64)
+    sign = np.where(np.signbit(v), 0x80, 0).astype(np.int64)
+    a = np.abs(v)
+    code = np.zeros(a.shape, np.int64)
+    sub = a < 2.0 ** -6
+    # subnormal range: multiples of 2^-9 (a count of 8 is the smallest normal, code 0x08)
+    code = np.where(sub, np.rint(np.where(sub, a, 0.0) / 2.0 ** -9).astype(np.int64), code)
+    # normal range: a = f * 2^ex with f in [0.5, 1) -> exponent ex - 1, 3 mantissa bits
+    with np.errstate(divide="ignore", invalid="ignore"):
+        _, ex = np.frexp(np.where(sub | ~np.isfinite(a), 1.0, a))
+    e = ex.astype(np.int64) - 1
+    q = np.rint(np.where(sub | ~np.isfinite(a), 8.0, a / np.exp2(e - 3.0))).astype(np.int64)  # in [8, 16]
+    carry = q == 16
+    e = np.where(carry, e + 1, e)
+    q = np.where(carry, 8, q)
+    normal = ((e + 7) << 3) | (q - 8)
+    normal = np.where((e > 8) | ((e == 8) & (q > 14)) | np.isinf(a), 0x7E, normal)
+    code = np.where(sub, code, normal)
+    code = code | sign
+    code = np.where(np.isnan(v), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def cache_token_slot(c, b: int, j: int) -> Tuple[object, int]:
+    """Where token j of batch row b is stored: (index into the first axis, token slot)."""
+    if c.page_size:
+        return int(c.page_table[b, j // c.page_size]), j % c.page_size
+    return b, j
+
+
+def cache_rows_f64(inp, b: int, h: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Keys and values of (b, kv head h) as exact float64 [N, d], read from the cache as stored."""
+    c = getattr(inp, "cache", None)
+    if c is None:
+        return bf16_to_f64(inp.K[b, h]), bf16_to_f64(inp.V[b, h])
+    if c.page_size:
+        rows = [cache_token_slot(c, b, j) for j in range(c.N)]
+        Kc = np.stack([c.K[p, h, slot] for p, slot in rows])
+        Vc = np.stack([c.V[p, h, slot] for p, slot in rows])
+    else:
+        Kc, Vc = c.K[b, h], c.V[b, h]
+    if c.dtype == "bf16":
+        return bf16_to_f64(Kc), bf16_to_f64(Vc)
+    if c.dtype == "fp8_e4m3":
+        return e4m3_to_f64(Kc) * float(c.k_scale[b, h]), e4m3_to_f64(Vc) * float(c.v_scale[b, h])
+    raise ValueError(f"unknown cache dtype {c.dtype}")
+
+
+def append_token(c, b: int, j: int, k_bits: np.ndarray, v_bits: np.ndarray) -> None:
+    """Write one new token (bf16 K and V rows [Hkv, d]) into the cache at position j, in place:
+    bf16 caches store the bits as they are, fp8 caches the E4M3 codes of value / scale."""
+    p, slot = cache_token_slot(c, b, j)
+    for h in range(c.Hkv):
+        if c.dtype == "bf16":
+            c.K[p, h, slot] = k_bits[h]
+            c.V[p, h, slot] = v_bits[h]
+        else:
+            c.K[p, h, slot] = quantize_e4m3(bf16_to_f64(k_bits[h]).astype(np.float32), c.k_scale[b, h])
+            c.V[p, h, slot] = quantize_e4m3(bf16_to_f64(v_bits[h]).astype(np.float32), c.v_scale[b, h])
+
+
+def decode_loop(steps, cache):
+    """A run of decode steps (``DecodeSteps``) over ``cache`` (a ``KVCache``, copied first).
+
+    Step s appends token s of every batch row at position pos + 1 and computes the hybrid step
+    for a query at that position.  Returns (per-step {(b, h, 0): RowResult}, final cache)."""
+    c = cache.copy()
+    pos = steps.start.pos[:, -1].astype(np.int64).copy()
+    results = []
+    for s in range(steps.Qf.shape[0]):
+        pos += 1
+        for b in range(pos.shape[0]):
+            append_token(c, b, int(pos[b]), steps.K_new[s, b], steps.V_new[s, b])
+        inp = replace(steps.start, Qf=steps.Qf[s], Qs=steps.Qs[s], pos=pos[:, None].astype(np.int32), cache=c)
+        results.append(step_rows(inp))
+    return results, c
 
 
 def rank_pool(s: np.ndarray) -> np.ndarray:
@@ -172,7 +286,7 @@ def step_rows(inp, rows: Optional[Iterable[Tuple[int, int, int]]] = None,
     evaluating sparse attention (used to score a different but valid index set).
     """
     B, Hq, T, d = inp.Qf.shape
-    Hkv, N = inp.K.shape[1], inp.K.shape[2]
+    Hkv = inp.dims["Hkv"]
     G = Hq // Hkv
     scale = softmax_scale(d)
     if rows is None:
@@ -183,8 +297,7 @@ def step_rows(inp, rows: Optional[Iterable[Tuple[int, int, int]]] = None,
         by_head.setdefault((b, h), []).append(t)
     out: Dict[Tuple[int, int, int], RowResult] = {}
     for (b, h), ts in by_head.items():
-        Kh = bf16_to_f64(inp.K[b, h])
-        Vh = bf16_to_f64(inp.V[b, h])
+        Kh, Vh = cache_rows_f64(inp, b, h)
         heads = [hq for hq in range(Hq) if kv_head_of(hq, G) == h]
         for t in ts:
             pos = int(inp.pos[b, t])

@@ -293,3 +293,9 @@ ALL_PINS = [
     pin_window_and_count,
     pin_collapse_to_full_attention,
 ]
+
+
+# the stored-cache readers (fp8, paged, decode loop) have their own pins
+from tests.cache_pins import CACHE_PINS  # noqa: E402
+
+ALL_PINS = ALL_PINS + CACHE_PINS
