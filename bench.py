@@ -7,10 +7,16 @@ T=1, k=4096, W=512), the configuration the sparse-attention queries/s and HBM GB
 metric is quoted on.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--impl reference]
+                    [--workloads batched,prefill,...|none]
 
 Under torchrun (N > 1) every rank runs an independent replica of the workload on its own
 GPU (the step has no cross-GPU exchange); timing is the max over ranks.  Prints one JSON
 line on rank 0.  ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+
+On one GPU the same line also carries a ``workloads`` block: the other benchmark shapes
+(batched decode, chunked prefill, 1M-token decode at T = 1 and 16) and the headline shapes
+with the cache stored as FP8 E4M3 or in a paged pool, each with its step time, queries/s,
+roofline, clocks and a bounded CPU-oracle baseline.
 """
 from __future__ import annotations
 
@@ -34,13 +40,31 @@ L2_BYTES = 126 * 1000 * 1000
 L2_FLUSH_BYTES = 256 << 20
 
 
-def kv_bytes(w):
-    return 2 * w.B * w.Hkv * w.N * w.d * 2
+# Workloads the default run measures besides the headline one: the other benchmark shapes and
+# the headline shapes with the cache stored as FP8 E4M3 or in a paged pool.
+#   name -> (shape, cache dtype, page size)
+EXTRA_WORKLOADS = {
+    "batched": ("batched", "bf16", 0),
+    "prefill": ("prefill", "bf16", 0),
+    "1m_t1": ("1m_t1", "bf16", 0),
+    "1m_t16": ("1m_t16", "bf16", 0),
+    "long_fp8": ("long", "fp8_e4m3", 0),
+    "long_paged": ("long", "bf16", 64),
+    "1m_t1_fp8": ("1m_t1", "fp8_e4m3", 0),
+}
 
 
-def kv_fits_l2(w):
+def elem_bytes(kv_dtype):
+    return 1 if kv_dtype == "fp8_e4m3" else 2
+
+
+def kv_bytes(w, kv_dtype="bf16"):
+    return 2 * w.B * w.Hkv * w.N * w.d * elem_bytes(kv_dtype)
+
+
+def kv_fits_l2(w, kv_dtype="bf16"):
     """K and V together no larger than L2: the timed steps then flush L2 in between."""
-    return kv_bytes(w) <= L2_BYTES
+    return kv_bytes(w, kv_dtype) <= L2_BYTES
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -66,14 +90,15 @@ def flop_model(w):
     return 4.0 * w.B * w.Hq * w.d * visible
 
 
-def byte_model(w):
+def byte_model(w, kv_dtype="bf16"):
     """Algorithmic bytes per step.
 
     literal: K read once + the gathered K/V rows of the selection (the metric's formula);
     minimum: K and V read once + gathered rows + Q in, O/LSE/idx out.
-    kv_once: K and V read once -- the algorithmic bytes of the full-attention kernel."""
+    kv_once: K and V read once -- the algorithmic bytes of the full-attention kernel.
+    A cache row is d elements of 2 bytes (bf16) or 1 byte (FP8 E4M3)."""
     B, Hq, Hkv, d, N, T, k, W = w.B, w.Hq, w.Hkv, w.d, w.N, w.T, w.k, w.W
-    kv_row = d * 2
+    kv_row = d * elem_bytes(kv_dtype)
     k_bytes = B * Hkv * N * kv_row
     sel = 0
     for t in range(T):
@@ -197,19 +222,27 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
 
-def oracle_rows(w):
-    from long_context_sparse_hs2_b200.inputs import generate
+def oracle_rows(w, kv=("bf16", 0)):
+    from dataclasses import replace
+
+    from long_context_sparse_hs2_b200.inputs import bf16_cache, fp8_e4m3_cache, generate, paged_cache
 
     inp = generate(w)
+    kv_dtype, page_size = kv
+    if kv_dtype != "bf16" or page_size:
+        c = fp8_e4m3_cache(inp.K, inp.V) if kv_dtype == "fp8_e4m3" else bf16_cache(inp)
+        if page_size:
+            c = paged_cache(c, page_size, seed=w.seed, spare_pages=0)
+        inp = replace(inp, cache=c)
     rows = [(b, h, t) for t in range(w.T) for b in range(w.B) for h in range(w.Hkv)]
     return inp, rows
 
 
-def oracle_time(w, budget_s, inp_rows=None):
+def oracle_time(w, budget_s, inp_rows=None, kv=("bf16", 0)):
     """Time the fp64 oracle on a bounded sample of the workload's selection rows."""
     import oracle.hs2_oracle as O
 
-    inp, rows = inp_rows or oracle_rows(w)
+    inp, rows = inp_rows or oracle_rows(w, kv)
     done, t0 = 0, time.perf_counter()
     for r in rows:
         O.step_rows(inp, [r])
@@ -265,30 +298,50 @@ def cores():
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def run_gpu(args, rank, world, local_rank, dist):
+def run_gpu(w, kv_dtype, page_size, steps, warmup, e2e_steps, local_rank, dist):
+    """Time `steps` hs2 steps of workload w (cache stored as kv_dtype, paged if page_size) on
+    this rank's GPU, after `warmup` untimed ones; e2e_steps > 0 also times the public call with
+    host buffers and the copies inside the timed region."""
     import numpy as np
     import torch
     from long_context_sparse_hs2_b200 import build, hs2
-    from long_context_sparse_hs2_b200.inputs import generate
+    from long_context_sparse_hs2_b200.inputs import bf16_cache, fp8_e4m3_cache, generate, paged_cache
 
     build.build()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = workload(args.workload)
     inp = generate(w)
 
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    Qf, Qs, K, V = to_dev(inp.Qf), to_dev(inp.Qs), to_dev(inp.K), to_dev(inp.V)
+    Qf, Qs = to_dev(inp.Qf), to_dev(inp.Qs)
     pos = torch.from_numpy(inp.pos).to(dev)
-    dims = hs2.dims_of(Qf, K, w.k, w.W)
-    ws = hs2.alloc_workspace(dims, dev)
+    cache = None
+    if kv_dtype == "bf16" and not page_size:
+        K, V = to_dev(inp.K), to_dev(inp.V)
+        dims = hs2.dims_of(Qf, K, w.k, w.W)
+        ws = hs2.alloc_workspace(dims, dev)
+    else:
+        c = fp8_e4m3_cache(inp.K, inp.V) if kv_dtype == "fp8_e4m3" else bf16_cache(inp)
+        if page_size:
+            c = paged_cache(c, page_size, seed=w.seed, spare_pages=0)
+        t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+        kv = (to_dev(c.K), to_dev(c.V)) if kv_dtype == "bf16" else (t(c.K), t(c.V))
+        cache = hs2.KVCache(K=kv[0], V=kv[1], N=c.N, dtype=c.dtype, k_scale=t(c.k_scale), v_scale=t(c.v_scale),
+                            page_size=c.page_size, page_table=t(c.page_table))
+        del c
+        dims = hs2.dims_kv(Qf, cache, w.k, w.W)
+        ws = hs2.alloc_workspace_kv(dims, cache, dev)
+    del inp
     out = hs2.alloc_step_outputs(dims, dev)
     stream = torch.cuda.Stream(device=dev)
 
     def one_step():
-        hs2.step(Qf, Qs, K, V, pos, k=w.k, W=w.W, out=out, ws=ws, stream=stream)
+        if cache is None:
+            hs2.step(Qf, Qs, K, V, pos, k=w.k, W=w.W, out=out, ws=ws, stream=stream)
+        else:
+            hs2.step_kv(Qf, Qs, cache, pos, k=w.k, W=w.W, out=out, ws=ws, stream=stream)
 
     def barrier():
         if dist is not None:
@@ -296,7 +349,7 @@ def run_gpu(args, rank, world, local_rank, dist):
 
     # K and V smaller than L2: write a buffer larger than L2 between timed steps, outside the
     # events, so that no step finds the previous step's data in L2
-    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if kv_fits_l2(w) else None
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if kv_fits_l2(w, kv_dtype) else None
 
     def timed(n):
         torch.cuda.synchronize(dev)
@@ -321,7 +374,7 @@ def run_gpu(args, rank, world, local_rank, dist):
         return sum(e0.elapsed_time(e1) for e0, e1 in evs)
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             one_step()
     torch.cuda.synchronize(dev)
     assert hs2.read_device_status(ws, stream) == 0, "device status bits set during warm-up"
@@ -329,49 +382,117 @@ def run_gpu(args, rank, world, local_rank, dist):
     # main timed region (headline number), clocks sampled meanwhile
     l0 = hs2.launch_count()
     with ClockSampler(local_rank) as clk:
-        ms = timed(args.steps)
+        ms = timed(steps)
     launches = hs2.launch_count() - l0
     clocks = clk.summary()
 
     # traced timed region: per-kernel CUDA-event durations on the launch stream
     hs2.trace_enable(True)
-    ms_traced = timed(args.steps)
+    ms_traced = timed(steps)
     kern = hs2.trace_collect()
     hs2.trace_enable(False)
+    assert hs2.read_device_status(ws, stream) == 0, "device status bits set during the timed region"
 
-    # end to end through the public API with host buffers (pinned), copies inside the timed region
-    host_in = {n: t.cpu().pin_memory() for n, t in (("Qf", Qf), ("Qs", Qs), ("K", K), ("V", V), ("pos", pos))}
-    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
-    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in out.as_dict().items()}
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    ms_e2e, h2d, d2h = None, 0, 0
+    if e2e_steps > 0:
+        # end to end through the public API with host buffers (pinned), copies inside the timed region
+        host_in = {n: t.cpu().pin_memory() for n, t in (("Qf", Qf), ("Qs", Qs), ("K", K), ("V", V), ("pos", pos))}
+        dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+        host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in out.as_dict().items()}
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
 
-    def e2e_step():
-        for n in dev_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        hs2.step(dev_in["Qf"], dev_in["Qs"], dev_in["K"], dev_in["V"], dev_in["pos"], k=w.k, W=w.W, out=out,
-                 ws=ws, stream=stream)
-        for n, t in out.as_dict().items():
-            host_out[n].copy_(t, non_blocking=True)
+        def e2e_step():
+            for n in dev_in:
+                dev_in[n].copy_(host_in[n], non_blocking=True)
+            hs2.step(dev_in["Qf"], dev_in["Qs"], dev_in["K"], dev_in["V"], dev_in["pos"], k=w.k, W=w.W, out=out,
+                     ws=ws, stream=stream)
+            for n, t in out.as_dict().items():
+                host_out[n].copy_(t, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        e2e_step()
-        torch.cuda.synchronize(dev)
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
+        with torch.cuda.stream(stream):
             e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-    ms_e2e = e0.elapsed_time(e1)
+            torch.cuda.synchronize(dev)
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        assert hs2.read_device_status(ws, stream) == 0, "device status bits set during the end-to-end region"
 
     ms = max_over_ranks(ms, dist, dev)
-    ms_e2e = max_over_ranks(ms_e2e, dist, dev)
-    assert hs2.read_device_status(ws, stream) == 0, "device status bits set during the timed region"
     return dict(w=w, ms=ms, ms_traced=ms_traced, ms_e2e=ms_e2e, kern=kern, launches=launches, clocks=clocks,
                 h2d=h2d, d2h=d2h, dims=dims)
+
+
+def kernel_table(r, steps):
+    return {k: {"avg_us": 1000.0 * v[0] / v[1], "launches": v[1], "share": v[0] / max(r["ms_traced"], 1e-9)}
+            for k, v in r["kern"].items()}
+
+
+def roofline(w, kv_dtype, kern, peaks, peak_src, name):
+    """Roofline of the dominant kernel (the full-attention sweep) from its live CUDA-event time."""
+    bm = byte_model(w, kv_dtype)
+    top = max((k for k in kern if k.startswith("full_attn") or k == "umma_attn"), key=lambda k: kern[k]["avg_us"],
+              default=None)
+    if top is None:
+        return None
+    secs = kern[top]["avg_us"] * 1e-6
+    if top == "umma_attn":
+        # many query rows per kv head on the tcgen05 tensor cores: the sweep is a dense contraction
+        achieved = flop_model(w) / secs / 1e12
+        return {"bound": "tensor", "kernel": top, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peak_src} bf16 dense (MEASURED_PEAKS.json bf16_tflops, burst)",
+                "algorithmic_flops_per_launch": flop_model(w),
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
+    achieved = bm["kv_once"] / secs / 1e9
+    return {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((name, top)),
+            "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+            "algorithmic_bytes_per_launch": bm["kv_once"]}
+
+
+def hbm_block(w, kv_dtype, step_s, peaks):
+    bm = byte_model(w, kv_dtype)
+    return {"literal_bytes_per_step": bm["literal"], "literal_gbs": bm["literal"] / step_s / 1e9,
+            "literal_frac_of_8tbs": bm["literal"] / step_s / 1e9 / NOMINAL_HBM_GBS,
+            "min_bytes_per_step": bm["minimum"], "min_gbs": bm["minimum"] / step_s / 1e9,
+            "min_frac_of_8tbs": bm["minimum"] / step_s / 1e9 / NOMINAL_HBM_GBS,
+            "min_frac_of_measured": bm["minimum"] / step_s / 1e9 / peaks["hbm_gbs"]}
+
+
+def extra_workloads(args, names, peaks, peak_src):
+    """The `workloads` block: each extra workload timed on its own (one GPU, rank 0)."""
+    import torch
+
+    out = {}
+    for name in names:
+        shape, kv_dtype, page_size = EXTRA_WORKLOADS[name]
+        w = workload(shape)
+        t0 = time.perf_counter()
+        r = run_gpu(w, kv_dtype, page_size, args.extra_steps, args.warmup, 0, 0, None)
+        torch.cuda.empty_cache()
+        step_s = r["ms"] / 1000.0 / args.extra_steps
+        kern = kernel_table(r, args.extra_steps)
+        entry = {"workload": shape, "kv_cache": kv_dtype + (f", paged ({page_size}-token pages)" if page_size else ""),
+                 "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "T": w.T, "k": w.k, "W": w.W,
+                 "steps": args.extra_steps, "ms_per_step": step_s * 1000.0,
+                 "value": w.B * w.T / step_s, "unit": "queries/s",
+                 "roofline": roofline(w, kv_dtype, kern, peaks, peak_src, name),
+                 "hbm": hbm_block(w, kv_dtype, step_s, peaks), "kernels": kern, "clocks": r["clocks"],
+                 "l2": "flush between steps" if kv_fits_l2(w, kv_dtype) else "no flush (K/V exceed L2)"}
+        if not args.no_cpu_baseline:
+            qps_cpu, el, sample = oracle_time(w, args.extra_cpu_budget, kv=(kv_dtype, page_size))
+            entry["cpu_baseline"] = {"value": qps_cpu, "unit": "queries/s", "cores": cores(), "kind": "oracle",
+                                     "sample": sample, "seconds": el}
+        entry["wall_s"] = time.perf_counter() - t0
+        out[name] = entry
+    return out
 
 
 def main():
@@ -384,7 +505,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default=",".join(EXTRA_WORKLOADS),
+                    help="comma-separated extra workloads timed after the headline one (one GPU), or 'none'")
+    ap.add_argument("--extra-steps", type=int, default=20)
+    ap.add_argument("--extra-cpu-budget", type=float, default=3.0, help="seconds of oracle time per extra workload")
     args = ap.parse_args()
+    if args.workloads != "none":
+        unknown = [x for x in args.workloads.split(",") if x and x not in EXTRA_WORKLOADS]
+        if unknown:
+            ap.error(f"unknown workloads {unknown}; choose from {sorted(EXTRA_WORKLOADS)}")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -420,7 +549,7 @@ def main():
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
     try:
-        r = run_gpu(args, rank, world, local_rank, dist)
+        r = run_gpu(w, "bf16", 0, args.steps, args.warmup, args.e2e_steps, local_rank, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
@@ -428,46 +557,23 @@ def main():
         return
 
     peaks, peak_src = load_peaks()
-    bm = byte_model(w)
     n = max(world, 1)
     step_s = r["ms"] / 1000.0 / args.steps
     qps = replica_throughput(n, w.B * w.T, args.steps, r["ms"])
     e2e_step_s = r["ms_e2e"] / 1000.0 / args.e2e_steps
-    kern = {k: {"avg_us": 1000.0 * v[0] / v[1], "launches": v[1], "share": v[0] / max(r["ms_traced"], 1e-9)}
-            for k, v in r["kern"].items()}
-    top = max((k for k in kern if k.startswith("full_attn") or k == "umma_attn"), key=lambda k: kern[k]["avg_us"],
-              default=None)
-    roof = None
-    if top is not None:
-        secs = kern[top]["avg_us"] * 1e-6
-        if w.T * (w.Hq // w.Hkv) > 16:
-            # many query rows per kv head: the full-attention pass is a dense contraction
-            achieved = flop_model(w) / secs / 1e12
-            roof = {"bound": "tensor", "kernel": top, "achieved": achieved, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                    "peak_source": f"{peak_src} bf16 dense (MEASURED_PEAKS.json bf16_tflops, burst)",
-                    "algorithmic_flops_per_launch": flop_model(w)}
-        else:
-            achieved = bm["kv_once"] / secs / 1e9
-            roof = {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((w.name, top)),
-                    "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                    "algorithmic_bytes_per_launch": bm["kv_once"]}
+    kern = kernel_table(r, args.steps)
     line = {
         "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_s * 1000.0, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q/K/V, needles, AR(1) drift)",
         "config": cfg,
-        "hbm": {"literal_bytes_per_step": bm["literal"], "literal_gbs": bm["literal"] / step_s / 1e9,
-                "literal_frac_of_8tbs": bm["literal"] / step_s / 1e9 / NOMINAL_HBM_GBS,
-                "min_bytes_per_step": bm["minimum"], "min_gbs": bm["minimum"] / step_s / 1e9,
-                "min_frac_of_8tbs": bm["minimum"] / step_s / 1e9 / NOMINAL_HBM_GBS,
-                "min_frac_of_measured": bm["minimum"] / step_s / 1e9 / peaks["hbm_gbs"]},
-        "roofline": roof,
+        "hbm": hbm_block(w, "bf16", step_s, peaks),
+        "roofline": roofline(w, "bf16", kern, peaks, peak_src, w.name),
         "kernels": kern,
         "traced_ms_per_step": r["ms_traced"] / args.steps,
-        "e2e": {"value": replica_throughput(n, w.B * w.T, args.e2e_steps, r["ms_e2e"]), "unit": "queries/s", "h2d_bytes_per_step": r["h2d"],
-                "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_step_s * 1000.0, "steps": args.e2e_steps},
+        "e2e": {"value": replica_throughput(n, w.B * w.T, args.e2e_steps, r["ms_e2e"]), "unit": "queries/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_step_s * 1000.0,
+                "steps": args.e2e_steps},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
@@ -475,6 +581,13 @@ def main():
         qps_cpu, el, sample = oracle_time(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": qps_cpu, "unit": "queries/s", "cores": cores(), "kind": "oracle",
                                 "sample": sample, "seconds": el}
+    # the other benchmark shapes and cache formats, one GPU only (a multi-GPU run times the
+    # headline workload alone)
+    extras = [x for x in args.workloads.split(",") if x] if args.workloads != "none" else []
+    if n == 1 and extras:
+        t0 = time.perf_counter()
+        line["workloads"] = extra_workloads(args, extras, peaks, peak_src)
+        line["workloads_wall_s"] = time.perf_counter() - t0
     print(json.dumps(line))
 
 

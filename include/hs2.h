@@ -87,6 +87,8 @@ typedef enum hs2_status {
 #define HS2_DEV_NONFINITE     0x4u  /* a selection score was NaN: ranked below every finite score */
 #define HS2_DEV_TIMEOUT       0x8u  /* a pipeline wait exceeded its bound: kernel gave up, outputs invalid */
 #define HS2_DEV_CAND_OVERFLOW 0x10u /* informational: top-k threshold bucket overflowed its buffer; slow exact path used */
+#define HS2_DEV_BAD_PAGE      0x20u /* a page id outside [0, num_pages) in the page table: its tokens read as zeros
+                                       (gathers skip them); hs2_kv_append skipped the token */
 
 /* Problem shape.  The attention scale is fixed to d^-1/2. */
 typedef struct hs2_dims {
@@ -133,9 +135,8 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, c
  * chunked prefill, multi-query decode) the full-attention and score sweeps run on the tcgen05
  * tensor cores.  Two environment variables change the execution plan (results are the same up
  * to rounding order; the workspace size depends on them, so query hs2_workspace_size under the
- * same environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles, and with one
- * query per batch row (T = 1) HS2_FUSED_DECODE=1 runs the step as a single cooperative kernel
- * when its grid fits on the device. */
+ * same environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles.  The plan,
+ * and so the workspace size, also follows the current device's SM count. */
 HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
                     const void* K, const void* V, const int32_t* pos,
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,
@@ -170,6 +171,94 @@ HS2_API hs2_status hs2_sparse_attn_static(const hs2_dims* dims, const void* Q_sp
                                           const void* V, const int32_t* pos, const int32_t* idx,
                                           const int32_t* cnt, void* O_sparse, float* LSE_sparse,
                                           void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * The KV cache in other storage formats and layouts, and the decode loop.
+ *
+ * The pages give the shared cache's size (2.69 GB at 1M tokens) without its storage precision
+ * ("HySparse2 od Xiaomi...", section "Co rikaji vysledky -- a co z nich neplyne"), and serving an
+ * agent's long context means a cache that grows by one token per decode step ("HySparse2 Cuts
+ * the Prefill Path for Tool-Using Agents", section "Tool Responses Turn Prefill Into the
+ * Bottleneck").  These entry points take the cache as a descriptor instead of two contiguous
+ * bf16 tensors: bf16 or FP8 E4M3 codes with per-(b, kv head) scales, contiguous or in a paged
+ * pool.  The method is unchanged: every stored token is first read back to its value (code x
+ * scale for FP8) and the four definitions at the top of this file apply to those values.
+ * ------------------------------------------------------------------------------------------- */
+
+typedef enum hs2_kv_dtype {
+    HS2_KV_BF16 = 0,      /* bfloat16 values */
+    HS2_KV_FP8_E4M3 = 1   /* FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+                             S.1111.111 is NaN); value = code x scale of the token's (b, kv head) */
+} hs2_kv_dtype;
+
+/* Where and how the shared cache is stored.  All pointers are device memory owned by the caller.
+ *  - dtype: hs2_kv_dtype.  Element size: 2 bytes (bf16) or 1 byte (FP8).
+ *  - page_size = 0: contiguous, K and V are [B][Hkv][N][d] (16-byte aligned).
+ *  - page_size > 0 (a power of two, 8 .. 65536): paged, K and V are pools
+ *    [num_pages][Hkv][page_size][d] (16-byte aligned) and token j of batch row b is stored in page
+ *    page_table[b * max_pages + j / page_size], at slot j % page_size.  max_pages >= ceil(N /
+ *    page_size); num_pages * Hkv * page_size < 2^31.  Pages may be shared between batch rows and
+ *    appear in any order.  A page id outside [0, num_pages) for a token the kernels read sets
+ *    HS2_DEV_BAD_PAGE, and the token reads as zeros (gathered keys are skipped).
+ *  - k_scale, v_scale: FP8 only, fp32 [B][Hkv]; NULL for bf16.
+ * K and V are const for every entry point except hs2_kv_append and hs2_decode_step, which write
+ * new tokens into them. */
+typedef struct hs2_kv_cache {
+    int32_t dtype;
+    int32_t page_size;
+    int32_t num_pages;
+    int32_t max_pages;
+    void* K;
+    void* V;
+    const int32_t* page_table;
+    const float* k_scale;
+    const float* v_scale;
+} hs2_kv_cache;
+
+/* hs2_workspace_size for a cache described by `cache` (its dtype and layout change the plan).
+ * Returns 0 if the dims or the cache description are invalid or unsupported. */
+HS2_API size_t hs2_workspace_size_kv(const hs2_dims* dims, const hs2_kv_cache* cache);
+
+/* hs2_full_attn, hs2_select, hs2_sparse_attn and hs2_step over a cache descriptor; same
+ * arguments, layouts, results and status bits otherwise.  A bf16 contiguous descriptor gives
+ * exactly the calls above.  FP8 caches run the warp-level MMA path on f16 operands (every E4M3
+ * value is exact in f16; queries are scaled by a power of two per row into the f16 range); FP8
+ * and paged caches run 128-row query tiles on the warp-level MMA sweeps, not tcgen05. */
+HS2_API hs2_status hs2_full_attn_kv(const hs2_dims* dims, const void* Q_full, const hs2_kv_cache* cache,
+                                    const int32_t* pos, void* O_full, float* LSE_full, void* ws, size_t ws_bytes,
+                                    void* stream);
+HS2_API hs2_status hs2_select_kv(const hs2_dims* dims, const void* Q_full, const hs2_kv_cache* cache,
+                                 const float* LSE_full, const int32_t* pos, int32_t* idx, int32_t* cnt, void* ws,
+                                 size_t ws_bytes, void* stream);
+HS2_API hs2_status hs2_sparse_attn_kv(const hs2_dims* dims, const void* Q_sparse, const hs2_kv_cache* cache,
+                                      const int32_t* pos, const int32_t* idx, const int32_t* cnt, void* O_sparse,
+                                      float* LSE_sparse, void* ws, size_t ws_bytes, void* stream);
+HS2_API hs2_status hs2_step_kv(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
+                               const hs2_kv_cache* cache, const int32_t* pos, void* O_full, void* O_sparse,
+                               float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Writes new tokens into the cache: for every (b, kv head, t), the bf16 rows K_new[b][h][t][:] and
+ * V_new[b][h][t][:] ([B][Hkv][T][d]) become token pos[b][t] of the cache -- stored as they are
+ * (bf16) or as the E4M3 code of value / scale (one fp32 division, rounded to nearest even,
+ * magnitudes past 448 saturating to 448) for an FP8 cache.  A pos outside [0, N) (HS2_DEV_BAD_POS)
+ * or an unmapped page (HS2_DEV_BAD_PAGE) skips that token.  ws: at least 256 bytes (the status
+ * word, cleared by the call).  Two (b, t) naming the same token: one of them wins. */
+HS2_API hs2_status hs2_kv_append(const hs2_dims* dims, const hs2_kv_cache* cache, const void* K_new,
+                                 const void* V_new, const int32_t* pos, void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step of the loop (T = 1): for every batch row b, the new token (K_new/V_new
+ * [B][Hkv][1][d], bf16) is written into the cache at position pos[b] + 1 as hs2_kv_append does,
+ * pos[b] is advanced to that position on the device, and the hybrid step (hs2_step_kv) runs
+ * for a query at that position.  pos (int32 [B], device) is the loop's state: on entry the
+ * newest cached position of each row (-1 for an empty row), on exit the new one.  Nothing
+ * is read or written by the host, so a CUDA graph of one call replays the loop step after step.
+ * A row whose cache is full (pos[b] + 1 >= N) sets HS2_DEV_BAD_POS, appends nothing, keeps
+ * pos[b], and its step runs at position N - 1.  ws: hs2_workspace_size_kv(dims, cache) bytes. */
+HS2_API hs2_status hs2_decode_step(const hs2_dims* dims, const hs2_kv_cache* cache, const void* Q_full,
+                                   const void* Q_sparse, const void* K_new, const void* V_new, int32_t* pos,
+                                   void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx,
+                                   int32_t* cnt, void* ws, size_t ws_bytes, void* stream);
 
 /* Copies the device status word out of ws and waits for the stream (the only synchronising
  * call).  *bits receives the HS2_DEV_* bits; returns HS2_ERR_DEVICE if any bit other than

@@ -1,5 +1,4 @@
-// The full-attention sweep of one CTA, shared by the standalone full-attention kernel and
-// the fused decode-step kernel (sm_100a).
+// The full-attention sweep of one CTA (sm_100a), and the TMA producer the score sweep shares.
 //
 // Split-K flash-decode: a CTA owns one row block (the G query heads of one kv head for TQ
 // consecutive queries = 16*RT MMA rows) and one contiguous range of 64-key tiles.  A
@@ -32,10 +31,11 @@ __device__ __forceinline__ int clamp_pos(int p, int N, unsigned* status) {
     return p;
 }
 
-// Shared-memory layout of the streaming kernels (after 1 KB alignment).
-template <int D, int STAGES, int TENSORS>
+// Shared-memory layout of the streaming kernels (after 1 KB alignment).  EB: bytes per cache
+// element (2 for bf16, 1 for FP8 E4M3).
+template <int D, int STAGES, int TENSORS, int EB = 2>
 struct StreamSmem {
-    static constexpr int kTileBytes = kKeyTile * D * 2;                 // one tensor, one tile
+    static constexpr int kTileBytes = kKeyTile * D * EB;                // one tensor, one tile
     static constexpr int kStageBytes = TENSORS * kTileBytes;
     static constexpr int kRingBytes = STAGES * kStageBytes;
     static constexpr int kBarOff = kRingBytes;                           // full[STAGES], empty[STAGES]
@@ -43,12 +43,49 @@ struct StreamSmem {
     static constexpr int kBytes = kMiscOff + 16 + 128 * 4 + 1024;        // + alignment slack
 };
 
+// Issues the TMA loads of one tile (keys j0 .. j0 + 63 of kv slice bh = b*Hkv + h) of one tensor
+// into dst, completing on bar.  Contiguous caches take one 3-D box per 64-dim half (bf16) or one
+// box (FP8); a paged pool takes one 4-D box per page the tile touches (per half for bf16), at the
+// page's slot range.  Page ids come from the page table; one outside [0, num_pages), or a page
+// index past the table's row, loads zeros and flags HS2_DEV_BAD_PAGE (keys past pos are never
+// used, so the tail of a row's last tile may be unmapped).
+template <int D, bool FP8>
+__device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const KvSrc& kv,
+                                             int j0, int bh, int Hkv, uint64_t pol, unsigned* status) {
+    constexpr int kHalves = FP8 ? 1 : D / 64;
+    constexpr int kRowBytes = FP8 ? D : 128;    // bytes of one key row inside a half
+    constexpr int kHalfBytes = kKeyTile * kRowBytes;
+    if (kv.page_shift < 0) {
+#pragma unroll
+        for (int hb = 0; hb < kHalves; ++hb) tma_load_3d(dst + hb * kHalfBytes, map, bar, hb * 64, j0, bh, pol);
+        return;
+    }
+    const int ps = 1 << kv.page_shift;
+    const int box = ps < kKeyTile ? ps : kKeyTile;
+    const int b = bh / Hkv, h = bh % Hkv;
+    for (int r = 0; r < kKeyTile; r += box) {
+        const int j = j0 + r;
+        const int pi = j >> kv.page_shift;
+        int page = pi < kv.max_pages ? kv.page_table[static_cast<int64_t>(b) * kv.max_pages + pi] : -1;
+        if (page < 0 || page >= kv.num_pages) {
+            if (pi < kv.max_pages) {
+                pdl_wait();  // the status word is cleared by the call's first kernel
+                set_status(status, HS2_DEV_BAD_PAGE);
+            }
+            page = -1;  // whole box out of range: zeros
+        }
+#pragma unroll
+        for (int hb = 0; hb < kHalves; ++hb)
+            tma_load_4d(dst + hb * kHalfBytes + r * kRowBytes, map, bar, hb * 64, j & (ps - 1), h, page, pol);
+    }
+}
+
 // Producer side of the TMA ring: stream tiles [t_begin, t_begin + nt) of kv slice bh.
-template <int D, int STAGES, int TENSORS>
+template <int D, int STAGES, int TENSORS, bool FP8>
 __device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* ring, uint64_t* full,
-                              uint64_t* empty, volatile int* abort_flag, int t_begin, int nt, int bh,
-                              unsigned* status, bool stream) {
-    using L = StreamSmem<D, STAGES, TENSORS>;
+                              uint64_t* empty, volatile int* abort_flag, int t_begin, int nt, int bh, int Hkv,
+                              const KvSrc& kv, unsigned* status, bool stream) {
+    using L = StreamSmem<D, STAGES, TENSORS, FP8 ? 1 : 2>;
     const uint64_t pol = stream ? l2_evict_first() : l2_evict_normal();
     prefetch_tensormap(tmK);
     if (TENSORS == 2) prefetch_tensormap(tmV);
@@ -63,13 +100,8 @@ __device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, ui
         mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
         const int j0 = (t_begin + i) * kKeyTile;
         uint8_t* dst = ring + stage * L::kStageBytes;
-#pragma unroll
-        for (int half = 0; half < D / 64; ++half) {
-            tma_load_3d(dst + half * (kKeyTile * 128), tmK, &full[stage], half * 64, j0, bh, pol);
-            if (TENSORS == 2)
-                tma_load_3d(dst + L::kTileBytes + half * (kKeyTile * 128), tmV, &full[stage], half * 64, j0, bh,
-                            pol);
-        }
+        load_kv_tile<D, FP8>(dst, tmK, &full[stage], kv, j0, bh, Hkv, pol, status);
+        if (TENSORS == 2) load_kv_tile<D, FP8>(dst + L::kTileBytes, tmV, &full[stage], kv, j0, bh, Hkv, pol, status);
         ++issued;
     }
     // Drain: wait (bounded) for the last load issued into every stage, so no copy is still
@@ -86,13 +118,13 @@ __device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, ui
 // base-2 logits, and writes the split partial of every row of the block.  Returns false if a
 // pipeline wait ran out (HS2_DEV_TIMEOUT is then set).  *t_range receives the tile range.
 // Ends with the block synchronised; the ring is free again afterwards.
-template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS>
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8>
 __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttnArgs& a,
                                            uint8_t* smem, int split, int unit, int2* t_range) {
     constexpr int NKS = NC / RT;          // warps sharing one row tile (each a key slice)
     constexpr int KW = kKeyTile / NKS;    // keys per warp per tile
     static_assert(NC % RT == 0 && KW % 16 == 0, "bad warp split");
-    using L = StreamSmem<D, STAGES, 2>;
+    using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
     uint8_t* ring = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
     uint64_t* empty = full + STAGES;
@@ -124,7 +156,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     const int nt = t_end - t_begin;
     *t_range = make_int2(t_begin, t_end);
 
-    OnlineSoftmax<D> st;
+    OnlineSoftmax<D, FP8> st;
     st.init();
     const int rt = warp % RT, ks = warp / RT;
     const int g = lane >> 2, c = lane & 3;
@@ -135,15 +167,19 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
         return (b * a.Hq + h * a.G + (r % a.G)) * a.T + t;
     };
 
+    const float kscale = FP8 ? a.kv.k_scale[bh] : 1.f;
+    const float vscale = FP8 ? a.kv.v_scale[bh] : 1.f;
     if (warp == NC) {
         if (lane == 0)
-            produce_tiles<D, STAGES, 2>(tmK, tmV, ring, full, empty, abort_flag, t_begin, nt, bh, a.status,
-                                        a.stream_kv != 0);
+            produce_tiles<D, STAGES, 2, FP8>(tmK, tmV, ring, full, empty, abort_flag, t_begin, nt, bh, a.Hkv, a.kv,
+                                             a.status, a.stream_kv != 0);
         __syncwarp();
     } else {
-        QTile<D> q;
+        QTileOf<D, FP8> q;
         const int rq_lo = row_q(r_lo), rq_hi = row_q(r_hi);
         q.load(a.Q, rq_lo >= 0 ? static_cast<int64_t>(rq_lo) * D : -1, rq_hi >= 0 ? static_cast<int64_t>(rq_hi) * D : -1);
+        const float f_lo = logit_factor<D, FP8>(q, 0, a.scale_log2, kscale);
+        const float f_hi = logit_factor<D, FP8>(q, 1, a.scale_log2, kscale);
         const int p_lo = s_pos[r_lo], p_hi = s_pos[r_hi];
         const int key0 = ks * KW;
         float* lg_lo = nullptr;
@@ -165,8 +201,23 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             if (*abort_flag) break;
             const uint32_t kbase = smem_u32(ring + stage * L::kStageBytes);
             const uint32_t vbase = kbase + L::kTileBytes;
+            const int tile_j0 = (t_begin + i) * kKeyTile;
+            const bool past_end = tile_j0 + key0 + KW - 1 > jmax;
+            if (past_end) {
+                // Keys past the CTA's last position are masked (P = 0), but their cache slots may hold
+                // anything (an unwritten cache, a paged pool's unused slots): 0 x NaN would poison O.
+                // Zero this warp's V rows there; only the warp itself reads them.
+                constexpr int CH = D * (FP8 ? 1 : 2) / 16;
+                uint8_t* vtile = ring + stage * L::kStageBytes + L::kTileBytes;
+                for (int e = lane; e < KW * CH; e += 32) {
+                    const int r = key0 + e / CH;
+                    if (tile_j0 + r > jmax)
+                        *reinterpret_cast<uint4*>(vtile + kv_chunk_offset<D, FP8>(r, e % CH)) = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
             float sc[KW / 8][4];
-            qk_tile<D, KW>(q, kbase, key0, sc);
+            qk_any<D, KW, FP8>(q, kbase, key0, sc);
             const int jb = (t_begin + i) * kKeyTile + key0 + 2 * c;
 #pragma unroll
             for (int n = 0; n < KW / 8; ++n) {
@@ -174,7 +225,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
                 for (int e = 0; e < 4; ++e) {
                     const int j = jb + n * 8 + (e & 1);
                     const int p = (e < 2) ? p_lo : p_hi;
-                    const float v = sc[n][e] * a.scale_log2;
+                    const float v = sc[n][e] * ((e < 2) ? f_lo : f_hi);
                     sc[n][e] = (j <= p) ? v : -INFINITY;
                     if (KEEP_LOGITS && j <= p) {
                         float* lg = (e < 2) ? lg_lo : lg_hi;
@@ -183,6 +234,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
                 }
             }
             st.template update<KW>(sc, vbase, key0);
+            if (past_end) fence_async_smem();  // the zeros are ordered before the next TMA write
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
         }
@@ -194,10 +246,10 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     const PartialRef out{a.part_ml + static_cast<int64_t>(split) * (a.B * a.Hq * a.T),
                          a.part_acc + static_cast<int64_t>(split) * (a.B * a.Hq * a.T) * D};
     if (NKS == 1) {
-        if (warp < NC) store_partial<D>(st, out, [&](int r) { return row_q(rt * 16 + r); });
+        if (warp < NC) store_partial<D, FP8>(st, out, [&](int r) { return row_q(rt * 16 + r); }, vscale);
     } else {
         float* red = reinterpret_cast<float*>(ring);  // the ring is idle now
-        if (warp < NC) stash_state<D, NKS>(st, ks, red + rt * merge_floats<D, NKS>());
+        if (warp < NC) stash_state<D, NKS, FP8>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
         __syncthreads();
         // threads of the CTA split evenly over the RT tiles
         const int per = blockDim.x / RT;

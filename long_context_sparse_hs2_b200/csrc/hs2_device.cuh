@@ -91,6 +91,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
     }
 }
 
+// Makes this thread's ordinary shared-memory stores visible to the async proxy (TMA, tensor
+// core) before a following barrier arrive.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ------------------------------------------------------------------ inter-CTA barrier (co-resident CTAs only)
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -169,6 +173,17 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// 4-D tiled load (paged pool [num_pages][Hkv][page_size][d]: c0 = element, c1 = slot in the page,
+// c2 = kv head, c3 = page).  An out-of-range coordinate reads as zeros.
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -210,6 +225,29 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A(16x16, row) * B(16x8, col) + D, fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two fp32 -> packed f16x2 (round to nearest even); lo goes to the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two FP8 E4M3 codes (the low byte first) -> f16x2, exact (every E4M3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(r) : "r"(two_codes));
+    return r;
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); lo goes to the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
@@ -236,6 +274,27 @@ __device__ __forceinline__ uint32_t tile_chunk_offset(int row, int chunk16) {
     const int half = chunk16 >> 3;
     const int c = chunk16 & 7;
     return static_cast<uint32_t>(half * (kKeyTile * 128) + row * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// FP8 E4M3 tiles hold one D-byte row per key: D = 128 uses the same 128-byte swizzled rows as a
+// 64-dim bf16 half (TMA CU_TENSOR_MAP_SWIZZLE_128B); D = 64 uses 64-byte rows with the 64-byte
+// swizzle (16-byte chunk c of row r stored at chunk c ^ ((r >> 1) & 3), as TMA writes with
+// CU_TENSOR_MAP_SWIZZLE_64B).  chunk16 indexes 16-byte chunks (16 dims) of the row.
+template <int D>
+__device__ __forceinline__ uint32_t fp8_chunk_offset(int row, int chunk16) {
+    if constexpr (D == 128)
+        return static_cast<uint32_t>(row * 128 + ((chunk16 ^ (row & 7)) << 4));
+    else
+        return static_cast<uint32_t>(row * 64 + ((chunk16 ^ ((row >> 1) & 3)) << 4));
+}
+
+// Byte offset of 16-byte chunk `chunk16` of key `row` in a K/V tile of the cache's element type.
+template <int D, bool FP8>
+__device__ __forceinline__ uint32_t kv_chunk_offset(int row, int chunk16) {
+    if constexpr (FP8)
+        return fp8_chunk_offset<D>(row, chunk16);
+    else
+        return tile_chunk_offset(row, chunk16);
 }
 
 // ------------------------------------------------------------------ top-k keys

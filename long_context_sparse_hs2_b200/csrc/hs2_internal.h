@@ -15,7 +15,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kKeyTile = 64;                      // keys per K/V shared-memory tile
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bound on any single pipeline wait (2 s)
-constexpr int kSMs = 148;            // B200 streaming multiprocessors
 constexpr int kHistBins = 2048;      // top-k histogram buckets (see score_bin)
 constexpr int kTopkChunk = 4096;     // pool keys per CTA in the histogram / emit passes
 constexpr int kMetaInts = 8;
@@ -25,13 +24,28 @@ constexpr int kMetaInts = 8;
 //   kMetaDef / kMetaCand: emit counters (adjacent, 8-byte aligned: reserved together);
 //   kMetaDone: score/histogram CTAs finished
 //   kMetaSelDone: selection CTAs finished;     kMetaSparseDone: sparse-attention CTAs finished
-//   kMetaBarrier: the fused decode step's per-row barrier counter
+//   kMetaBarrier: unused
 enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDef = 2, kMetaCand = 3, kMetaDone = 4, kMetaSelDone = 5,
                 kMetaSparseDone = 6, kMetaBarrier = 7 };  // kMetaDef/kMetaCand share one 8-byte word
 constexpr int kSmemCand = 4096;      // candidates the final select keeps in shared memory
 constexpr int kMaxKW = 1 << 22;      // largest supported k + W
 constexpr int kSparseMaxC4 = 4096;         // most selected keys one sparse-attention CTA takes
-constexpr int kRowsPerCtaTopk = 4 * kSMs;  // from this many selection rows on, one top-k CTA per row
+constexpr int kRowsPerCtaTopkPerSM = 4;   // from 4 x (SMs) selection rows on, one top-k CTA per row
+
+// How the kernels find a token's K/V row in the cache (see hs2_kv_cache in hs2.h).
+//   contiguous: row (b*Hkv + h)*N + j of [B][Hkv][N][d]
+//   paged:      row (page*Hkv + h)*page_size + j % page_size of the pool, page =
+//               page_table[b*max_pages + j / page_size]; a page id outside [0, num_pages)
+//               (or a page index past max_pages) reads as zeros and flags HS2_DEV_BAD_PAGE
+// fp8: rows hold E4M3 codes (d bytes); k_scale/v_scale[b*Hkv + h] turn codes into values.
+struct KvSrc {
+    int fp8;
+    int page_shift;              // log2(page_size), or -1 for the contiguous layout
+    int max_pages, num_pages;
+    const int32_t* page_table;   // [B][max_pages]
+    const float* k_scale;        // [B*Hkv] (fp8 only)
+    const float* v_scale;
+};
 
 // Everything one call needs to know about shapes, grids and workspace offsets.
 struct Plan {
@@ -53,13 +67,24 @@ struct Plan {
     int64_t cand_cap;   // per-row capacity of the top-k candidate buffer
     int topk_ctas;      // CTAs per row of the multi-CTA top-k kernels (each takes every topk_ctas-th chunk)
     int64_t kstride;    // row stride (elements) of the score-key buffer: N rounded up to 64
-    bool fused;         // hs2_step runs the single fused decode-step kernel (T = 1, see k_decode.cu)
+    bool fp8;           // the cache holds FP8 E4M3 codes
+    bool paged;         // the cache is a paged pool
+    int page_size, max_pages, num_pages;
+    int sms;            // streaming multiprocessors of the device the plan was made for
     // workspace byte offsets
-    size_t off_status, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand,
+    size_t off_status, off_pos, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand,
         off_logits, zero_bytes, total;
 };
 
-bool make_plan(const hs2_dims* dims, Plan* p, hs2_status* why);
+// Cache description the plan depends on (dtype and layout only; pointers are checked per call).
+struct KvShape {
+    int fp8 = 0;
+    int page_size = 0;   // 0: contiguous
+    int max_pages = 0;
+    int num_pages = 0;
+};
+
+bool make_plan(const hs2_dims* dims, Plan* p, hs2_status* why, const KvShape& kv = KvShape());
 
 // ------------------------------------------------------------------ kernel arguments
 
@@ -79,6 +104,7 @@ struct AttnArgs {
     uint32_t* keys;        // [rows_kv][kstride] order-preserving score keys (score sweep only)
     int64_t kstride;
     int k;
+    KvSrc kv;              // cache layout / dtype (TMA producer and scales)
     unsigned* status;
 };
 
@@ -92,6 +118,7 @@ struct SparseArgs {
     int B, Hq, Hkv, T, N, G, kw;  // kw = k + W (row stride of idx)
     int C4, S4;
     int stages;            // gather ring depth (set by the launcher)
+    KvSrc kv;              // cache layout / dtype
     float scale_log2;
     float2* part_ml;       // [S4][rows_q]
     float* part_acc;       // [S4][rows_q][D]
@@ -100,38 +127,6 @@ struct SparseArgs {
     float* LSE;            // LSE_sparse [B][Hq][T]
     unsigned* status;
 };
-
-struct DecodeArgs {        // the fused decode step (T = 1)
-    AttnArgs attn;         // full sweep: Q_full, pos, shapes, full partials, kept logits
-    const uint16_t* Qs;    // Q_sparse [B][Hq][1][D]
-    const uint16_t* K;     // [B][Hkv][N][D] (gathered by the sparse phase)
-    const uint16_t* V;
-    int k, W;
-    float2* ps_ml;         // sparse partials [S1][rows_q]
-    float* ps_acc;         // [S1][rows_q][D]
-    unsigned* hist;        // [rows][kHistBins]
-    int* meta;             // [rows][kMetaInts]
-    unsigned long long* cand;  // [rows][cand_cap]
-    int64_t cand_cap;
-    int32_t* idx;          // [rows][k+W]
-    int32_t* cnt;          // [rows]
-    uint16_t* O_full;
-    float* LSE_full;
-    uint16_t* O_sparse;
-    float* LSE_sparse;
-};
-
-// Shared-memory plan of the fused decode step's phases after the sweep (byte offsets from the
-// 1 KB-aligned base; the sweep ring below is 96 KB).
-constexpr int kFusedLseOff = 0;          // 16 floats: per-head base-2 LSE
-constexpr int kFusedWbufOff = 1024;      // 256 floats: combine weights
-constexpr int kFusedHistOff = 2048;      // kHistBins u32 (phases A, B); then 2 x 64 gather slots (D)
-constexpr int kFusedKeysOff = 10240;     // this split's pool keys (u32), phases A and B
-constexpr int kFusedCandOff = 10240;     // phase C: candidates held in shared memory
-constexpr int kFusedRingOff = 32768;     // phase D: gather ring, 2 tiles of K and V
-constexpr int kFusedSmemCand = (kFusedRingOff - kFusedCandOff) / 8;
-constexpr int kFusedMaxKeys = (96 * 1024 - kFusedKeysOff) / 4;
-constexpr int kFusedMaxSlice = 4096;
 
 struct CombineArgs {
     const float2* part_ml;
@@ -180,10 +175,11 @@ void trace_mark(const char* name, cudaStream_t st, bool kernel = true);  // afte
 
 // ------------------------------------------------------------------ launch helper
 
-// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger).
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger) -- or, with
+// pdl = false, as an ordinary launch that starts only after everything before it completed.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args&&... args) {
+cudaError_t launch_pdl_opt(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                           Args&&... args) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -193,16 +189,41 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    return launch_pdl_opt(true, kern, grid, block, smem, st, static_cast<Args&&>(args)...);
 }
 
 // ------------------------------------------------------------------ launchers (return cudaGetLastError())
 
+int num_sms();  // streaming multiprocessors of the current device (queried once per device)
+
 cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st);  // clears ws[0, bytes) (normal launch)
 
+// New tokens into the cache (hs2_kv_append / hs2_decode_step).  pos_in[b*T + t] (+1 when advance)
+// is the token's position; with advance (T = 1) the position is also written to pos_out[b] and
+// pos_new[b].  Ordinary launch.
+struct AppendArgs {
+    const uint16_t* K_new;  // [B][Hkv][T][d] bf16
+    const uint16_t* V_new;
+    void* K;                // cache (contiguous or pool)
+    void* V;
+    KvSrc kv;
+    const int32_t* pos_in;
+    int32_t* pos_out;       // advance: the caller's pos, updated
+    int32_t* pos_new;       // advance: the position the step runs at (workspace copy)
+    int B, Hkv, T, N, d;
+    int advance;
+    unsigned* status;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
+
 cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
-                             cudaStream_t st);
+                             cudaStream_t st, bool pdl = true);  // pdl = false: an ordinary launch
 cudaError_t launch_umma_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                              cudaStream_t st);  // tensor maps with 128-key boxes
 cudaError_t launch_umma_score(const Plan& p, const CUtensorMap& tmK, const AttnArgs& a,
@@ -212,10 +233,6 @@ cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK
 cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st);
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st);
-// The fused decode step; returns cudaErrorCooperativeLaunchTooLarge if its grid cannot be
-// co-resident (the caller then runs the multi-kernel path).
-cudaError_t launch_decode_step(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a,
-                               cudaStream_t st);
 cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st);
 cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st);
 

@@ -89,6 +89,7 @@ extern "C" hs2_status hs2_sparse_attn_static(const hs2_dims* dims, const void* Q
     sa.cnt = cnt;
     sa.B = p.B; sa.Hq = p.Hq; sa.Hkv = p.Hkv; sa.T = p.T; sa.N = p.N; sa.G = p.G; sa.kw = p.k + p.W;
     sa.C4 = p.C4; sa.S4 = p.S4;
+    sa.kv.page_shift = -1;  // contiguous bf16 cache
     sa.scale_log2 = kLog2e / sqrtf(static_cast<float>(p.d));
     sa.part_ml = reinterpret_cast<float2*>(base + off_ml);
     sa.part_acc = reinterpret_cast<float*>(base + off_acc);

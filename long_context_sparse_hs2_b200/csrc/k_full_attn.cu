@@ -1,4 +1,5 @@
-// Full-attention layer and selection-score sweeps over the shared KV cache (sm_100a).
+// Full-attention layer and selection-score sweeps over the shared KV cache (sm_100a), for bf16
+// or FP8 E4M3 caches, contiguous or paged (the TMA producer in attn_sweep.cuh).
 //
 // full_attn_kernel: the split-K flash-decode sweep (attn_sweep.cuh) as a kernel of its own.
 //
@@ -20,7 +21,7 @@ namespace hs2 {
 
 // ====================================================================== full attention
 
-template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS>
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8>
 __global__ void __launch_bounds__((NC + 1) * 32)
     full_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const AttnArgs a) {
@@ -34,7 +35,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             a.zero[i] = make_uint4(0, 0, 0, 0);
     }
     int2 range;
-    full_sweep<D, RT, NC, STAGES, KEEP_LOGITS>(&tmK, &tmV, a, smem, blockIdx.x, blockIdx.y, &range);
+    full_sweep<D, RT, NC, STAGES, KEEP_LOGITS, FP8>(&tmK, &tmV, a, smem, blockIdx.x, blockIdx.y, &range);
     // The sweep reads nothing its predecessor writes, but it must not complete before the
     // predecessor does (later kernels rely on that chain).
     pdl_wait();
@@ -47,12 +48,12 @@ __global__ void __launch_bounds__((NC + 1) * 32)
 // query m).  A lane's two accumulator rows m and m+8 are then two heads of one query, so the max
 // over the G heads is one local max plus log2(G/2) lane shuffles (instead of log2(G)).
 
-template <int D, int RT, int NC, int STAGES>
+template <int D, int RT, int NC, int STAGES, bool FP8>
 __global__ void __launch_bounds__((NC + 1) * 32)
     score_sweep_kernel(const __grid_constant__ CUtensorMap tmK, const AttnArgs a) {
     constexpr int NKS = NC / RT;
     constexpr int KW = kKeyTile / NKS;
-    using L = StreamSmem<D, STAGES, 1>;
+    using L = StreamSmem<D, STAGES, 1, FP8 ? 1 : 2>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* ring = smem;
@@ -105,8 +106,8 @@ __global__ void __launch_bounds__((NC + 1) * 32)
 
     if (warp == NC) {
         if (lane == 0)
-            produce_tiles<D, STAGES, 1>(&tmK, &tmK, ring, full, empty, abort_flag, t_begin, nt, bh, a.status,
-                                        a.stream_kv != 0);
+            produce_tiles<D, STAGES, 1, FP8>(&tmK, &tmK, ring, full, empty, abort_flag, t_begin, nt, bh, a.Hkv, a.kv,
+                                             a.status, a.stream_kv != 0);
         __syncwarp();
     }
     const int rt = warp % RT, ks = warp / RT;
@@ -130,9 +131,12 @@ __global__ void __launch_bounds__((NC + 1) * 32)
     const bool writer = G >= 2 ? (m_lo < Q8) : true;
     bool nonfinite = false;
     if (warp < NC) {
-        QTile<D> q;
+        QTileOf<D, FP8> q;
         const int rq_lo = row_q(tq_lo, g_lo), rq_hi = row_q(tq_hi, g_hi);
         q.load(a.Q, rq_lo >= 0 ? static_cast<int64_t>(rq_lo) * D : -1, rq_hi >= 0 ? static_cast<int64_t>(rq_hi) * D : -1);
+        const float kscale = FP8 ? a.kv.k_scale[bh] : 1.f;
+        const float f2[2] = {logit_factor<D, FP8>(q, 0, a.scale_log2, kscale),
+                             logit_factor<D, FP8>(q, 1, a.scale_log2, kscale)};
         pdl_wait();  // LSE_full comes from the previous kernel
         // base-2 LSE of the two rows (+inf for padding rows so their scores are -inf)
         const float lse_lo = rq_lo >= 0 ? a.lse[rq_lo] * kLog2e : INFINITY;
@@ -152,7 +156,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             if (*abort_flag) break;
             const uint32_t kbase = smem_u32(ring + stage * L::kStageBytes);
             float sc[KW / 8][4];
-            qk_tile<D, KW>(q, kbase, key0, sc);
+            qk_any<D, KW, FP8>(q, kbase, key0, sc);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             const int jb = (t_begin + i) * kKeyTile + key0 + 2 * c;
@@ -160,7 +164,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             for (int n = 0; n < KW / 8; ++n) {
                 float v[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) v[e] = sc[n][e] * a.scale_log2 - ((e < 2) ? lse_lo : lse_hi);
+                for (int e = 0; e < 4; ++e) v[e] = sc[n][e] * f2[e >> 1] - ((e < 2) ? lse_lo : lse_hi);
                 if (G >= 2) {
                     v[0] = nan_max(v[0], v[2]);  // heads g and g + G/2 of the same query
                     v[1] = nan_max(v[1], v[3]);
@@ -214,28 +218,30 @@ cudaError_t set_smem(Kern kern, int bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int D, int RT, bool KEEP>
+template <int D, int RT, bool KEEP, bool FP8>
 cudaError_t full_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool pdl) {
     constexpr int NC = RT >= 8 ? 8 : 4;
-    constexpr int STAGES = D == 128 ? 3 : 6;
-    using L = StreamSmem<D, STAGES, 2>;
-    auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP>;
+    // ring of 96 KB (bf16: 3 stages at d = 128, 6 at d = 64; FP8 twice as many), two CTAs per SM
+    constexpr int STAGES = (D == 128 ? 3 : 6) * (FP8 ? 2 : 1);
+    using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
+    static_assert(L::kRingBytes >= RT * merge_floats<D, NC / RT>() * 4, "merge scratch must fit in the ring");
+    auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP, FP8>;
     cudaError_t e = set_smem(kern, L::kBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S1, p.B * p.Hkv * p.QB);
-    e = launch_pdl(kern, grid, dim3((NC + 1) * 32), L::kBytes, st, tmK, tmV, a);
+    e = launch_pdl_opt(pdl, kern, grid, dim3((NC + 1) * 32), L::kBytes, st, tmK, tmV, a);
     trace_mark(KEEP ? "full_attn_keep_logits" : "full_attn", st);
     return e;
 }
 
-template <int D, int RT>
+template <int D, int RT, bool FP8>
 cudaError_t score_sweep_variant(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a,
                                 cudaStream_t st) {
     constexpr int NC = RT >= 8 ? 8 : 4;
-    constexpr int STAGES = D == 128 ? 6 : 12;
-    using L = StreamSmem<D, STAGES, 1>;
-    auto kern = score_sweep_kernel<D, RT, NC, STAGES>;
+    constexpr int STAGES = (D == 128 ? 6 : 12) * (FP8 ? 2 : 1);
+    using L = StreamSmem<D, STAGES, 1, FP8 ? 1 : 2>;
+    auto kern = score_sweep_kernel<D, RT, NC, STAGES, FP8>;
     cudaError_t e = set_smem(kern, L::kBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(splits, p.B * p.Hkv * p.QB);
@@ -247,24 +253,28 @@ cudaError_t score_sweep_variant(const Plan& p, int splits, const CUtensorMap& tm
 }  // namespace
 
 cudaError_t launch_full_attn(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool pdl) {
     const bool keep = a.logits != nullptr;
-#define HS2_FA(D_, RT_)                                                                                  \
-    if (p.d == D_ && p.RT == RT_)                                                                        \
-        return (keep && RT_ == 1) ? full_attn_variant<D_, RT_, (RT_ == 1)>(p, tmK, tmV, a, st)           \
-                                  : full_attn_variant<D_, RT_, false>(p, tmK, tmV, a, st);
-    HS2_FA(64, 1) HS2_FA(64, 2) HS2_FA(64, 4) HS2_FA(64, 8)
-    HS2_FA(128, 1) HS2_FA(128, 2) HS2_FA(128, 4) HS2_FA(128, 8)
+#define HS2_FA(D_, RT_, F_)                                                                              \
+    if (p.d == D_ && p.RT == RT_ && p.fp8 == F_)                                                         \
+        return (keep && RT_ == 1) ? full_attn_variant<D_, RT_, (RT_ == 1), F_>(p, tmK, tmV, a, st, pdl)  \
+                                  : full_attn_variant<D_, RT_, false, F_>(p, tmK, tmV, a, st, pdl);
+    HS2_FA(64, 1, false) HS2_FA(64, 2, false) HS2_FA(64, 4, false) HS2_FA(64, 8, false)
+    HS2_FA(128, 1, false) HS2_FA(128, 2, false) HS2_FA(128, 4, false) HS2_FA(128, 8, false)
+    HS2_FA(64, 1, true) HS2_FA(64, 2, true) HS2_FA(64, 4, true) HS2_FA(64, 8, true)
+    HS2_FA(128, 1, true) HS2_FA(128, 2, true) HS2_FA(128, 4, true) HS2_FA(128, 8, true)
 #undef HS2_FA
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK, const AttnArgs& a,
                                cudaStream_t st) {
-#define HS2_SS(D_, RT_) \
-    if (p.d == D_ && p.RT == RT_) return score_sweep_variant<D_, RT_>(p, splits, tmK, a, st);
-    HS2_SS(64, 1) HS2_SS(64, 2) HS2_SS(64, 4) HS2_SS(64, 8)
-    HS2_SS(128, 1) HS2_SS(128, 2) HS2_SS(128, 4) HS2_SS(128, 8)
+#define HS2_SS(D_, RT_, F_) \
+    if (p.d == D_ && p.RT == RT_ && p.fp8 == F_) return score_sweep_variant<D_, RT_, F_>(p, splits, tmK, a, st);
+    HS2_SS(64, 1, false) HS2_SS(64, 2, false) HS2_SS(64, 4, false) HS2_SS(64, 8, false)
+    HS2_SS(128, 1, false) HS2_SS(128, 2, false) HS2_SS(128, 4, false) HS2_SS(128, 8, false)
+    HS2_SS(64, 1, true) HS2_SS(64, 2, true) HS2_SS(64, 4, true) HS2_SS(64, 8, true)
+    HS2_SS(128, 1, true) HS2_SS(128, 2, true) HS2_SS(128, 4, true) HS2_SS(128, 8, true)
 #undef HS2_SS
     return cudaErrorInvalidValue;
 }
@@ -278,7 +288,7 @@ __global__ void __launch_bounds__(256) init_kernel(uint4* p, int64_t n) {
 
 cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st) {
     const int64_t n = static_cast<int64_t>(bytes / 16);
-    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(8 * kSMs, std::max<int64_t>(1, (n + 255) / 256)));
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(8 * num_sms(), std::max<int64_t>(1, (n + 255) / 256)));
     init_kernel<<<blocks, 256, 0, st>>>(static_cast<uint4*>(ws), n);
     trace_mark("init", st);
     return cudaGetLastError();

@@ -1,4 +1,5 @@
-// Sparse layer with KV Reuse: attention of Q_sparse over the selected keys only (sm_100a).
+// Sparse layer with KV Reuse: attention of Q_sparse over the selected keys only (sm_100a), from a
+// bf16 or FP8 E4M3 cache, contiguous or paged (the gather resolves each index to its pool row).
 //
 // Each sparse layer of a hybrid block reuses the preceding full-attention layer's KV
 // cache and its token selection ("HySparse2 od Xiaomi zkracuje zpracovani dlouheho
@@ -31,9 +32,9 @@ constexpr int kSparseTile = 2 * kKeyTile;  // keys per pipeline step: two 64-key
 
 constexpr int kSparseMaxStages = 3;  // ring depth for long rows; short rows use fewer (less smem)
 
-template <int D>
+template <int D, bool FP8>
 struct SparseSmem {
-    static constexpr int kTileBytes = kKeyTile * D * 2;    // one 64-key sub-tile of K (or V)
+    static constexpr int kTileBytes = kKeyTile * D * (FP8 ? 1 : 2);  // one 64-key sub-tile of K (or V)
     static constexpr int kSubBytes = 2 * kTileBytes;       // K + V of one sub-tile
     static constexpr int kStageBytes = 2 * kSubBytes;      // two sub-tiles = one 128-key step
     // After the main loop the ring is reused as scratch: the warps' softmax states are merged
@@ -60,25 +61,30 @@ __device__ __forceinline__ void cp_async_wait_upto(int pending) {
 }
 
 // Gathers the K and V rows of 128-key step `tile` into a stage: sub-tile u (keys 64u..64u+63
-// of the step) at u * kSubBytes, K then V, each in the swizzled 64-key tile layout.  Thread t
-// copies 16-byte chunk t mod (D/8) of rows t / (D/8), + 256/(D/8), ... of both sub-tiles, K and
-// V alike: one index load and one address per row for two copies.
-template <int D>
-__device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_idx, int tile, uint8_t* stage,
+// of the step) at u * kSubBytes, K then V, each in the swizzled 64-key tile layout of the cache's
+// element type.  Thread t copies 16-byte chunk t mod CH of rows t / CH, + 256/CH, ... of both
+// sub-tiles, K and V alike: one index load and one address per row for two copies.  s_row holds
+// the cache row of every slot (-1: empty or skipped); kv_base is added for a contiguous cache.
+template <int D, bool FP8>
+__device__ __forceinline__ void gather_tile(const SparseArgs& a, const int* s_row, int tile, uint8_t* stage,
                                             int64_t kv_base) {
-    constexpr int CH = D / 8;                       // 16-byte chunks per row
+    using L = SparseSmem<D, FP8>;
+    constexpr int RB = D * (FP8 ? 1 : 2);           // bytes per cache row
+    constexpr int CH = RB / 16;                     // 16-byte chunks per row
     constexpr int RSTEP = kSparseThreads / CH;      // rows covered per pass
     const int c16 = threadIdx.x % CH, r0 = threadIdx.x / CH;
+    const uint8_t* Kb = reinterpret_cast<const uint8_t*>(a.K);
+    const uint8_t* Vb = reinterpret_cast<const uint8_t*>(a.V);
 #pragma unroll
     for (int sub = 0; sub < 2; ++sub) {
 #pragma unroll
         for (int rr = r0; rr < kKeyTile; rr += RSTEP) {
-            const int j = s_idx[tile * kSparseTile + sub * kKeyTile + rr];
-            const int64_t off = (kv_base + (j >= 0 ? j : 0)) * D + c16 * 8;
+            const int j = s_row[tile * kSparseTile + sub * kKeyTile + rr];
+            const int64_t off = (kv_base + (j >= 0 ? j : 0)) * RB + c16 * 16;
             const uint32_t nbytes = j >= 0 ? 16u : 0u;
-            uint8_t* dst = stage + sub * SparseSmem<D>::kSubBytes + tile_chunk_offset(rr, c16);
-            cp_async16(dst, a.K + off, nbytes);
-            cp_async16(dst + SparseSmem<D>::kTileBytes, a.V + off, nbytes);
+            uint8_t* dst = stage + sub * L::kSubBytes + kv_chunk_offset<D, FP8>(rr, c16);
+            cp_async16(dst, Kb + off, nbytes);
+            cp_async16(dst + L::kTileBytes, Vb + off, nbytes);
         }
     }
 }
@@ -108,9 +114,9 @@ __device__ __forceinline__ void finish_row(const SparseArgs& a, int row, int64_t
 
 // MINB: CTAs per SM the register allocation must allow (2 for one-step CTAs, whose ring is a
 // single 64 KB stage; 1 for the deep-ring variant, which also gets the registers to avoid spills).
-template <int D, int MINB>
+template <int D, int MINB, bool FP8>
 __global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const SparseArgs a) {
-    using L = SparseSmem<D>;
+    using L = SparseSmem<D, FP8>;
     constexpr int KW = 16;  // keys per warp per step: warps 0-3 take sub-tile 0, warps 4-7 sub-tile 1
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -148,7 +154,8 @@ __global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const
     }
 
     const int ntl = (nk + kSparseTile - 1) / kSparseTile;
-    bool bad = false;
+    const bool paged = a.kv.page_shift >= 0;
+    bool bad = false, bad_page = false;
     for (int i = tid; i < ntl * kSparseTile; i += kSparseThreads) {
         int j = -1;
         if (i < nk) {
@@ -156,26 +163,39 @@ __global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const
             if (j < 0 || j > pos) {
                 bad = true;
                 j = -1;
+            } else if (paged) {  // the token's row in the page pool
+                const int page = a.kv.page_table[static_cast<int64_t>(b) * a.kv.max_pages + (j >> a.kv.page_shift)];
+                if (page < 0 || page >= a.kv.num_pages) {
+                    bad_page = true;
+                    j = -1;
+                } else {
+                    j = (page * a.Hkv + h) * (1 << a.kv.page_shift) + (j & ((1 << a.kv.page_shift) - 1));
+                }
             }
         }
         s_idx[i] = j;
     }
     if (__syncthreads_or(bad) && tid == 0) set_status(a.status, HS2_DEV_BAD_INDEX);
+    if (__syncthreads_or(bad_page) && tid == 0) set_status(a.status, HS2_DEV_BAD_PAGE);
 
-    const int64_t kv_base = static_cast<int64_t>(bh) * a.N;
+    const int64_t kv_base = paged ? 0 : static_cast<int64_t>(bh) * a.N;
     const int prime = min(ntl, stages);
     for (int i = 0; i < prime; ++i) {
-        gather_tile<D>(a, s_idx, i, smem + i * L::kStageBytes, kv_base);
+        gather_tile<D, FP8>(a, s_idx, i, smem + i * L::kStageBytes, kv_base);
         cp_async_commit();
     }
 
     const int g = lane >> 2, c = lane & 3;
-    QTile<D> q;
+    QTileOf<D, FP8> q;
     {
         const int r0 = row_q(g), r1 = row_q(g + 8);
         q.load(a.Q, r0 >= 0 ? static_cast<int64_t>(r0) * D : -1, r1 >= 0 ? static_cast<int64_t>(r1) * D : -1);
     }
-    OnlineSoftmax<D> st;
+    const float kscale = FP8 ? a.kv.k_scale[bh] : 1.f;
+    const float vscale = FP8 ? a.kv.v_scale[bh] : 1.f;
+    const float f_lo = logit_factor<D, FP8>(q, 0, a.scale_log2, kscale);
+    const float f_hi = logit_factor<D, FP8>(q, 1, a.scale_log2, kscale);
+    OnlineSoftmax<D, FP8> st;
     st.init();
     const int sub = warp >> 2;
     const int key0 = (warp & 3) * KW;
@@ -186,34 +206,34 @@ __global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const
         const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes + sub * L::kSubBytes);
         const uint32_t vbase = kbase + L::kTileBytes;
         float sc[KW / 8][4];
-        qk_tile<D, KW>(q, kbase, key0, sc);
+        qk_any<D, KW, FP8>(q, kbase, key0, sc);
         const int slot0 = i * kSparseTile + sub * kKeyTile + key0 + 2 * c;
 #pragma unroll
         for (int nn = 0; nn < KW / 8; ++nn)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const bool ok = s_idx[slot0 + nn * 8 + (e & 1)] >= 0;
-                sc[nn][e] = ok ? sc[nn][e] * a.scale_log2 : -INFINITY;
+                sc[nn][e] = ok ? sc[nn][e] * (e < 2 ? f_lo : f_hi) : -INFINITY;
             }
         st.template update<KW>(sc, vbase, key0);
         __syncthreads();  // everyone is done with this stage before it is refilled
         if (i + stages < ntl) {
-            gather_tile<D>(a, s_idx, i + stages, smem + stage * L::kStageBytes, kv_base);
+            gather_tile<D, FP8>(a, s_idx, i + stages, smem + stage * L::kStageBytes, kv_base);
             cp_async_commit();
         }
     }
     st.finish_rows();
     float* red = reinterpret_cast<float*>(smem);
-    stash_state<D, kSparseWarps>(st, warp, red);
+    stash_state<D, kSparseWarps, FP8>(st, warp, red, vscale);
     __syncthreads();
     merge_states<D, kSparseWarps>(red, tid, kSparseThreads, out, row_q);
     finish_row<D>(a, row, out_rows_q_base(a, b, h, t), smem);
 }
 
-template <int D, int MINB>
+template <int D, int MINB, bool FP8>
 cudaError_t sparse_variant(const Plan& p, const SparseArgs& x, cudaStream_t st) {
-    auto kern = sparse_attn_kernel<D, MINB>;
-    const int bytes = SparseSmem<D>::bytes(x.stages, p.C4);
+    auto kern = sparse_attn_kernel<D, MINB, FP8>;
+    const int bytes = SparseSmem<D, FP8>::bytes(x.stages, p.C4);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3(p.S4, static_cast<unsigned>(p.rows_kv)), dim3(kSparseThreads), bytes, st, x);
@@ -221,12 +241,16 @@ cudaError_t sparse_variant(const Plan& p, const SparseArgs& x, cudaStream_t st) 
     return e;
 }
 
+template <int D, bool FP8>
+cudaError_t sparse_dispatch(const Plan& p, const SparseArgs& x, cudaStream_t st) {
+    return x.stages == 1 ? sparse_variant<D, 2, FP8>(p, x, st) : sparse_variant<D, 1, FP8>(p, x, st);
+}
+
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st) {
     SparseArgs x = a;
     x.stages = std::min(kSparseMaxStages, (p.C4 + kSparseTile - 1) / kSparseTile);
-    const bool one_step = x.stages == 1;
-    if (p.d == 128) return one_step ? sparse_variant<128, 2>(p, x, st) : sparse_variant<128, 1>(p, x, st);
-    return one_step ? sparse_variant<64, 2>(p, x, st) : sparse_variant<64, 1>(p, x, st);
+    if (p.d == 128) return p.fp8 ? sparse_dispatch<128, true>(p, x, st) : sparse_dispatch<128, false>(p, x, st);
+    return p.fp8 ? sparse_dispatch<64, true>(p, x, st) : sparse_dispatch<64, false>(p, x, st);
 }
 
 }  // namespace hs2

@@ -17,7 +17,8 @@
 //   warps 0-3   softmax of stream 0 (thread = TMEM lane = tile row), warps 4-7 stream 1
 //   warp 8      TMA producer: K and V tiles of 128 keys into two 2-stage rings
 //   warp 9      allocates TMEM; one lane issues every tcgen05.mma and commit
-//   warps 10-11 idle after the prologue; with warps 8 and 9 they form the warpgroup that
+//   warps 10-11 zero the V rows of keys past the CTA's last position in its last tile (when
+//               that tile reaches past it); with warps 8 and 9 they form the warpgroup that
 //               hands registers to the softmax warpgroups (setmaxnreg)
 // TMEM (512 columns): stream s has S at columns 256s .. 256s+127 (fp32 logits; the bf16
 // probabilities P overwrite its first 64 columns) and O at 256s+128 .. 256s+128+D-1.
@@ -61,7 +62,7 @@ struct USmem {
     static constexpr int kKOff = 2 * kQBytes;
     static constexpr int kVOff = kKOff + kUStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kUStages * kTileBytes;
-    static constexpr int kNumBars = 4 * kUStages + 5;    // kfull, kempty, vfull, vempty, sfull[2], pfull[2], done
+    static constexpr int kNumBars = 4 * kUStages + 6;    // kfull, kempty, vfull, vempty, sfull[2], pfull[2], done, vfix
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kPosOff = kMiscOff + 16;        // row positions of both streams
     static constexpr int kBytes = kPosOff + 2 * kURows * 4 + 1024;  // + alignment slack
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
     uint64_t* sfull = bars + 4 * kUStages;
     uint64_t* pfull = sfull + 2;
     uint64_t* done = sfull + 4;
+    uint64_t* vfix = sfull + 5;  // the last V tile with its rows past the last position zeroed
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
     int* s_pos = reinterpret_cast<int*>(smem + L::kPosOff);
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < L::kNumBars; ++i) mbar_init(&bars[i], i >= 4 * kUStages + 2 && i < 4 * kUStages + 4
                                                                       ? kURows   // pfull: one arrival per row
-                                                                      : 1);
+                                                                      : (i == 4 * kUStages + 5 ? 64 : 1));  // vfix: warps 10-11
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -160,6 +162,10 @@ __global__ void __launch_bounds__(kUThreads, 1)
     const int nstep0 = split_keys ? (nt + 1) / 2 : nt;
     const int nstep1 = split_keys ? nt / 2 : nt;
     auto seq_of = [&](int s, int i) { return split_keys ? 2 * i + s : i; };
+    // The CTA's last tile reaches past its largest position: those keys are masked (P = 0), but
+    // their cache slots may hold anything (an unwritten cache), and 0 x NaN would poison O.  Warps
+    // 10-11 zero those V rows once the tile lands; the PV MMA of that tile waits for them.
+    const bool fix_last = nt > 0 && t_end == ntiles && ntiles * kUTile - 1 > jmax;
 
     if (warp >= 8) {
         reg_dealloc<kURegsOther>();
@@ -228,7 +234,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
             auto issue_pv = [&](int s, int i) -> bool {
                 if (!mbar_wait(&pfull[s], i & 1, a.status)) return false;
                 const int q = seq_of(s, i), st = q % kUStages;
-                if (!mbar_wait(&vfull[st], (q / kUStages) & 1, a.status)) return false;
+                if (fix_last && q == nt - 1) {
+                    if (!mbar_wait(vfix, 0, a.status)) return false;
+                } else if (!mbar_wait(&vfull[st], (q / kUStages) & 1, a.status)) {
+                    return false;
+                }
                 tc_fence_after();
                 const uint32_t vb = vb0 + st * L::kTileBytes;
 #pragma unroll
@@ -252,6 +262,25 @@ __global__ void __launch_bounds__(kUThreads, 1)
             if (!ok) *abort_flag = 1;
             umma_commit(done);
             mbar_wait(done, 0, a.status);  // nothing of this CTA is left in the tensor core
+        }
+        __syncwarp();
+    } else if (fix_last) {
+        // ------------------------------------------------------------ warps 10-11: zero the V rows
+        // of keys past jmax in the last tile (rows of 128 bytes in each 64-dim block)
+        const int q = nt - 1, st = q % kUStages;
+        const bool landed = mbar_wait(&vfull[st], (q / kUStages) & 1, a.status);
+        if (landed) {
+            uint8_t* vt = smem + L::kVOff + st * L::kTileBytes;
+            const int r0 = jmax + 1 - (t_begin + q) * kUTile;  // first row to clear, in [1, 127]
+            const int t = (warp - 10) * 32 + lane;
+            for (int e = t; e < (kUTile - r0) * (D / 8); e += 64) {
+                const int r = r0 + e / (D / 8), c = e % (D / 8);
+                *reinterpret_cast<uint4*>(vt + (c >> 3) * L::kBlock + r * 128 + (c & 7) * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_async_smem();  // visible to the tensor core before the arrive
+            mbar_arrive(vfix);
+        } else {
+            *abort_flag = 1;
         }
         __syncwarp();
     }

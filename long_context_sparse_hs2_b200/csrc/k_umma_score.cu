@@ -302,7 +302,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
                 for (int qq = 0; qq < 32 / G; ++qq) {
                     const float sv = head_max<G>(m + qq * G) * c2;
-                    nonfinite |= (sv != sv);
+                    // only keys that are stored count (past a query's pool the slot may hold anything)
+                    nonfinite |= (sv != sv) && (fast || j <= s_pl[qa0 + (32 * cq) / G + qq]);
                     key[qq] = score_key(sv);
                 }
                 uint32_t* kq = kp + static_cast<int64_t>((32 * cq) / G) * a.kstride;

@@ -7,7 +7,10 @@ step of the computation runs in the library's CUDA kernels; there is no CPU or
 PyTorch fallback, and a missing library is an error.
 
 Names mirror the C entry points: ``full_attn``, ``select``, ``sparse_attn``,
-``step``, ``workspace_size``, ``read_device_status``, ``status_string``.
+``step``, ``workspace_size``, ``read_device_status``, ``status_string``, and for a cache
+described by a ``KVCache`` (bf16 or FP8 E4M3, contiguous or paged) ``full_attn_kv``,
+``select_kv``, ``sparse_attn_kv``, ``step_kv``, ``workspace_size_kv``, ``kv_append`` and
+``decode_step``.
 """
 from __future__ import annotations
 
@@ -24,9 +27,14 @@ LIB_PATH = os.path.join(_HERE, "libhs2.so")
 HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUDA, HS2_ERR_DEVICE = range(6)
 DEV_BAD_POS, DEV_BAD_INDEX, DEV_NONFINITE, DEV_TIMEOUT, DEV_CAND_OVERFLOW = 0x1, 0x2, 0x4, 0x8, 0x10
 
+DEV_BAD_PAGE = 0x20
+KV_BF16, KV_FP8_E4M3 = 0, 1
+
 ENTRY_POINTS = ("hs2_workspace_size", "hs2_full_attn", "hs2_select", "hs2_sparse_attn", "hs2_step",
                 "hs2_read_device_status", "hs2_status_string", "hs2_trace_enable", "hs2_trace_collect",
-                "hs2_launch_count", "hs2_version", "hs2_sparse_attn_static")
+                "hs2_launch_count", "hs2_version", "hs2_sparse_attn_static", "hs2_workspace_size_kv",
+                "hs2_full_attn_kv", "hs2_select_kv", "hs2_sparse_attn_kv", "hs2_step_kv", "hs2_kv_append",
+                "hs2_decode_step")
 STATIC_SCRATCH_BYTES = 4 << 20  # HS2_STATIC_SCRATCH_BYTES
 
 
@@ -37,6 +45,14 @@ class Dims(ctypes.Structure):
 
     def as_tuple(self):
         return tuple(getattr(self, n) for n, _ in self._fields_)
+
+
+class KvCacheDesc(ctypes.Structure):
+    """``hs2_kv_cache``: storage format and layout of the shared KV cache."""
+
+    _fields_ = [("dtype", ctypes.c_int32), ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("max_pages", ctypes.c_int32), ("K", ctypes.c_void_p), ("V", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p)]
 
 
 class HS2Error(RuntimeError):
@@ -66,6 +82,18 @@ def lib() -> ctypes.CDLL:
     L.hs2_step.argtypes = [dp, vp, vp, vp, vp, i32p, vp, vp, f32p, f32p, i32p, i32p, vp, sz, vp]
     L.hs2_sparse_attn_static.argtypes = [dp, vp, vp, vp, i32p, i32p, i32p, vp, f32p, vp]
     L.hs2_sparse_attn_static.restype = ctypes.c_int
+    cp = ctypes.POINTER(KvCacheDesc)
+    L.hs2_workspace_size_kv.argtypes = [dp, cp]
+    L.hs2_workspace_size_kv.restype = sz
+    L.hs2_full_attn_kv.argtypes = [dp, vp, cp, i32p, vp, f32p, vp, sz, vp]
+    L.hs2_select_kv.argtypes = [dp, vp, cp, f32p, i32p, i32p, i32p, vp, sz, vp]
+    L.hs2_sparse_attn_kv.argtypes = [dp, vp, cp, i32p, i32p, i32p, vp, f32p, vp, sz, vp]
+    L.hs2_step_kv.argtypes = [dp, vp, vp, cp, i32p, vp, vp, f32p, f32p, i32p, i32p, vp, sz, vp]
+    L.hs2_kv_append.argtypes = [dp, cp, vp, vp, i32p, vp, sz, vp]
+    L.hs2_decode_step.argtypes = [dp, cp, vp, vp, vp, vp, i32p, vp, vp, f32p, f32p, i32p, i32p, vp, sz, vp]
+    for f in ("hs2_full_attn_kv", "hs2_select_kv", "hs2_sparse_attn_kv", "hs2_step_kv", "hs2_kv_append",
+              "hs2_decode_step"):
+        getattr(L, f).restype = ctypes.c_int
     L.hs2_read_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.hs2_status_string.argtypes = [ctypes.c_int]
     L.hs2_status_string.restype = ctypes.c_char_p
@@ -284,6 +312,209 @@ def step(Q_full, Q_sparse, K, V, pos, *, k: int, W: int, out: Optional[StepOutpu
         _check(lib().hs2_step(ctypes.byref(dm), _p(Q_full), _p(Q_sparse), _p(K), _p(V), _p(pos), _p(out.O_full),
                               _p(out.O_sparse), _p(out.LSE_full), _p(out.LSE_sparse), _p(out.idx), _p(out.cnt),
                               _p(ws), ws.numel(), _stream(stream, dev)), "hs2_step")
+    return out
+
+
+# ----------------------------------------------------------------------------- cache descriptors
+
+@dataclass
+class KVCache:
+    """The shared KV cache as stored (``hs2_kv_cache``).
+
+    dtype "bf16": K/V are bfloat16 tensors.  dtype "fp8_e4m3": K/V hold E4M3 codes (uint8 or
+    torch.float8_e4m3fn) and k_scale/v_scale (float32 [B, Hkv]) turn them into values.
+    page_size = 0: K/V are [B, Hkv, N, d].  page_size > 0: K/V are pools
+    [num_pages, Hkv, page_size, d] and page_table (int32 [B, max_pages]) maps token j of row b
+    to page page_table[b, j // page_size].  N is the number of token positions per row."""
+
+    K: torch.Tensor
+    V: torch.Tensor
+    N: int
+    dtype: str = "bf16"
+    k_scale: Optional[torch.Tensor] = None
+    v_scale: Optional[torch.Tensor] = None
+    page_size: int = 0
+    page_table: Optional[torch.Tensor] = None
+
+    @property
+    def Hkv(self) -> int:
+        return int(self.K.shape[1])
+
+    def tensors(self) -> Dict[str, torch.Tensor]:
+        out = dict(K=self.K, V=self.V, k_scale=self.k_scale, v_scale=self.v_scale, page_table=self.page_table)
+        return {k: v for k, v in out.items() if v is not None}
+
+    def check(self, B: int, d: int) -> None:
+        if self.dtype not in ("bf16", "fp8_e4m3"):
+            raise ValueError(f"unknown cache dtype {self.dtype}")
+        fp8 = self.dtype == "fp8_e4m3"
+        allowed = (torch.uint8, torch.float8_e4m3fn) if fp8 else (torch.bfloat16,)
+        Hkv = self.Hkv
+        if self.page_size:
+            npg = int(self.K.shape[0])
+            shape = (npg, Hkv, self.page_size, d)
+            if self.page_table is None:
+                raise ValueError("a paged cache needs page_table")
+            _need(self.page_table, "page_table", torch.int32, (B, int(self.page_table.shape[1])))
+        else:
+            shape = (B, Hkv, self.N, d)
+        for name in ("K", "V"):
+            t = getattr(self, name)
+            if t.dtype not in allowed:
+                raise TypeError(f"{name} must be one of {allowed} for a {self.dtype} cache, got {t.dtype}")
+            _need(t, name, t.dtype, shape)
+        if fp8:
+            for name in ("k_scale", "v_scale"):
+                t = getattr(self, name)
+                if t is None:
+                    raise ValueError(f"an fp8 cache needs {name}")
+                _need(t, name, torch.float32, (B, Hkv))
+
+    def desc(self) -> KvCacheDesc:
+        return KvCacheDesc(dtype=KV_FP8_E4M3 if self.dtype == "fp8_e4m3" else KV_BF16,
+                           page_size=int(self.page_size),
+                           num_pages=int(self.K.shape[0]) if self.page_size else 0,
+                           max_pages=int(self.page_table.shape[1]) if self.page_size else 0,
+                           K=_p(self.K), V=_p(self.V), page_table=_p(self.page_table), k_scale=_p(self.k_scale),
+                           v_scale=_p(self.v_scale))
+
+
+def dims_kv(Q: torch.Tensor, cache: KVCache, k: int, W: int) -> Dims:
+    B, Hq, T, d = Q.shape
+    return make_dims(B, Hq, cache.Hkv, T, cache.N, d, k, W)
+
+
+def workspace_size_kv(dims: Dims, cache: KVCache) -> int:
+    """Bytes of workspace the cache-descriptor entry points need (0 if unsupported)."""
+    desc = cache.desc()
+    return int(lib().hs2_workspace_size_kv(ctypes.byref(dims), ctypes.byref(desc)))
+
+
+def alloc_workspace_kv(dims: Dims, cache: KVCache, device) -> torch.Tensor:
+    n = workspace_size_kv(dims, cache)
+    if n == 0:
+        raise HS2Error(HS2_ERR_UNSUPPORTED, "workspace_size_kv")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _kv_call(where, Q, cache, k, W, ws, extra):
+    """Shape/device checks shared by the cache-descriptor calls; returns (dims, desc, device)."""
+    dm = dims_kv(Q, cache, k, W)
+    cache.check(dm.B, dm.d)
+    dev = device_of(where, Q=Q, ws=ws, **cache.tensors(), **{n: t for n, t in extra.items() if t is not None})
+    return dm, cache.desc(), dev
+
+
+def full_attn_kv(Q_full, cache: KVCache, pos, *, k: int = 0, W: int = 0, O_full=None, LSE_full=None, ws=None,
+                 stream=None):
+    """hs2_full_attn_kv: the full-attention layer over a cache descriptor."""
+    dm, desc, dev = _kv_call("full_attn_kv", Q_full, cache, k, W, ws, dict(pos=pos, O_full=O_full, LSE_full=LSE_full))
+    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
+    _need(Q_full, "Q_full", torch.bfloat16, (B, Hq, T, d))
+    _need(pos, "pos", torch.int32, (B, T))
+    with torch.cuda.device(dev):
+        O_full = torch.empty_like(Q_full) if O_full is None else O_full
+        LSE_full = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if LSE_full is None else LSE_full
+        ws = alloc_workspace_kv(dm, cache, dev) if ws is None else ws
+        _check(lib().hs2_full_attn_kv(ctypes.byref(dm), _p(Q_full), ctypes.byref(desc), _p(pos), _p(O_full),
+                                      _p(LSE_full), _p(ws), ws.numel(), _stream(stream, dev)), "hs2_full_attn_kv")
+    return O_full, LSE_full
+
+
+def select_kv(Q_full, cache: KVCache, LSE_full, pos, *, k: int, W: int, idx=None, cnt=None, ws=None, stream=None):
+    """hs2_select_kv: top-k + window over a cache descriptor."""
+    dm, desc, dev = _kv_call("select_kv", Q_full, cache, k, W, ws, dict(LSE_full=LSE_full, pos=pos, idx=idx, cnt=cnt))
+    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
+    _need(Q_full, "Q_full", torch.bfloat16, (B, Hq, T, d))
+    _need(LSE_full, "LSE_full", torch.float32, (B, Hq, T))
+    _need(pos, "pos", torch.int32, (B, T))
+    with torch.cuda.device(dev):
+        idx = torch.empty((B, Hkv, T, k + W), dtype=torch.int32, device=dev) if idx is None else idx
+        cnt = torch.empty((B, Hkv, T), dtype=torch.int32, device=dev) if cnt is None else cnt
+        ws = alloc_workspace_kv(dm, cache, dev) if ws is None else ws
+        _check(lib().hs2_select_kv(ctypes.byref(dm), _p(Q_full), ctypes.byref(desc), _p(LSE_full), _p(pos), _p(idx),
+                                   _p(cnt), _p(ws), ws.numel(), _stream(stream, dev)), "hs2_select_kv")
+    return idx, cnt
+
+
+def sparse_attn_kv(Q_sparse, cache: KVCache, pos, idx, cnt, *, k: int, W: int, O_sparse=None, LSE_sparse=None,
+                   ws=None, stream=None):
+    """hs2_sparse_attn_kv: the sparse layer (KV Reuse over idx/cnt) over a cache descriptor."""
+    dm, desc, dev = _kv_call("sparse_attn_kv", Q_sparse, cache, k, W, ws,
+                             dict(pos=pos, idx=idx, cnt=cnt, O_sparse=O_sparse, LSE_sparse=LSE_sparse))
+    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
+    _need(Q_sparse, "Q_sparse", torch.bfloat16, (B, Hq, T, d))
+    _need(pos, "pos", torch.int32, (B, T))
+    _need(idx, "idx", torch.int32, (B, Hkv, T, k + W))
+    _need(cnt, "cnt", torch.int32, (B, Hkv, T))
+    with torch.cuda.device(dev):
+        O_sparse = torch.empty_like(Q_sparse) if O_sparse is None else O_sparse
+        LSE_sparse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev) if LSE_sparse is None else LSE_sparse
+        ws = alloc_workspace_kv(dm, cache, dev) if ws is None else ws
+        _check(lib().hs2_sparse_attn_kv(ctypes.byref(dm), _p(Q_sparse), ctypes.byref(desc), _p(pos), _p(idx),
+                                        _p(cnt), _p(O_sparse), _p(LSE_sparse), _p(ws), ws.numel(),
+                                        _stream(stream, dev)), "hs2_sparse_attn_kv")
+    return O_sparse, LSE_sparse
+
+
+def step_kv(Q_full, Q_sparse, cache: KVCache, pos, *, k: int, W: int, out: Optional["StepOutputs"] = None, ws=None,
+            stream=None) -> "StepOutputs":
+    """hs2_step_kv: the whole hybrid step over a cache descriptor."""
+    outs = out.as_dict() if out is not None else {}
+    dm, desc, dev = _kv_call("step_kv", Q_full, cache, k, W, ws, dict(Q_sparse=Q_sparse, pos=pos, **outs))
+    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
+    _need(Q_full, "Q_full", torch.bfloat16, (B, Hq, T, d))
+    _need(Q_sparse, "Q_sparse", torch.bfloat16, (B, Hq, T, d))
+    _need(pos, "pos", torch.int32, (B, T))
+    with torch.cuda.device(dev):
+        out = alloc_step_outputs(dm, dev) if out is None else out
+        ws = alloc_workspace_kv(dm, cache, dev) if ws is None else ws
+        _check(lib().hs2_step_kv(ctypes.byref(dm), _p(Q_full), _p(Q_sparse), ctypes.byref(desc), _p(pos),
+                                 _p(out.O_full), _p(out.O_sparse), _p(out.LSE_full), _p(out.LSE_sparse), _p(out.idx),
+                                 _p(out.cnt), _p(ws), ws.numel(), _stream(stream, dev)), "hs2_step_kv")
+    return out
+
+
+def kv_append(cache: KVCache, K_new, V_new, pos, *, ws=None, stream=None) -> torch.Tensor:
+    """hs2_kv_append: K_new/V_new (bf16 [B, Hkv, T, d]) become tokens pos[b, t] of the cache.
+    Returns the status workspace (read it with read_device_status)."""
+    B, Hkv, T, d = K_new.shape
+    cache.check(B, d)
+    _need(K_new, "K_new", torch.bfloat16, (B, cache.Hkv, T, d))
+    _need(V_new, "V_new", torch.bfloat16, (B, cache.Hkv, T, d))
+    _need(pos, "pos", torch.int32, (B, T))
+    dev = device_of("kv_append", K_new=K_new, V_new=V_new, pos=pos, ws=ws, **cache.tensors())
+    dm = make_dims(B, cache.Hkv, cache.Hkv, T, cache.N, d, 0, 0)
+    desc = cache.desc()
+    with torch.cuda.device(dev):
+        ws = torch.empty(256, dtype=torch.uint8, device=dev) if ws is None else ws
+        _check(lib().hs2_kv_append(ctypes.byref(dm), ctypes.byref(desc), _p(K_new), _p(V_new), _p(pos), _p(ws),
+                                   ws.numel(), _stream(stream, dev)), "hs2_kv_append")
+    return ws
+
+
+def decode_step(Q_full, Q_sparse, cache: KVCache, K_new, V_new, pos, *, k: int, W: int,
+                out: Optional["StepOutputs"] = None, ws=None, stream=None) -> "StepOutputs":
+    """hs2_decode_step: append the new token at pos[b] + 1 (device-side pos advances) and run the
+    step for it.  Q_full/Q_sparse [B, Hq, 1, d], K_new/V_new [B, Hkv, 1, d] bf16, pos int32 [B]."""
+    outs = out.as_dict() if out is not None else {}
+    dm, desc, dev = _kv_call("decode_step", Q_full, cache, k, W, ws,
+                             dict(Q_sparse=Q_sparse, K_new=K_new, V_new=V_new, pos=pos, **outs))
+    B, Hq, Hkv, T, N, d, _, _ = dm.as_tuple()
+    if T != 1:
+        raise ValueError("decode_step takes one query per batch row (T = 1)")
+    _need(Q_full, "Q_full", torch.bfloat16, (B, Hq, 1, d))
+    _need(Q_sparse, "Q_sparse", torch.bfloat16, (B, Hq, 1, d))
+    _need(K_new, "K_new", torch.bfloat16, (B, Hkv, 1, d))
+    _need(V_new, "V_new", torch.bfloat16, (B, Hkv, 1, d))
+    _need(pos, "pos", torch.int32, (B,))
+    with torch.cuda.device(dev):
+        out = alloc_step_outputs(dm, dev) if out is None else out
+        ws = alloc_workspace_kv(dm, cache, dev) if ws is None else ws
+        _check(lib().hs2_decode_step(ctypes.byref(dm), ctypes.byref(desc), _p(Q_full), _p(Q_sparse), _p(K_new),
+                                     _p(V_new), _p(pos), _p(out.O_full), _p(out.O_sparse), _p(out.LSE_full),
+                                     _p(out.LSE_sparse), _p(out.idx), _p(out.cnt), _p(ws), ws.numel(),
+                                     _stream(stream, dev)), "hs2_decode_step")
     return out
 
 

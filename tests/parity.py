@@ -34,9 +34,9 @@ def assert_close_o(got, want, what=""):
     want = np.asarray(want, dtype=np.float64)
     err = np.abs(got - want)
     bound = O_ATOL + O_RTOL * np.abs(want)
-    bad = err > bound
+    bad = ~(err <= bound)  # NaN anywhere fails
     if bad.any():
-        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        i = np.unravel_index(np.argmax(np.where(np.isnan(err), np.inf, err - bound)), err.shape)
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements off; worst at {i}: got {got[i]} want {want[i]}")
 
 
@@ -75,3 +75,27 @@ def check_selection(idx_row: np.ndarray, cnt: int, row, tol: float = SCORE_TIE_T
         assert np.all(row.scores[missing] <= sk + tol), \
             f"dropped keys {missing[row.scores[missing] > sk + tol][:5]} beat the k-th score {sk}"
     return S
+
+
+def gpu_cache(c, device="cuda"):
+    """A generator-side KVCache (numpy) as the binding's KVCache (device tensors)."""
+    from long_context_sparse_hs2_b200 import hs2
+
+    def dev(a, dtype=None):
+        if a is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return t.to(device) if dtype is None else t.view(dtype).to(device)
+
+    kv_dtype = torch.bfloat16 if c.dtype == "bf16" else None
+    K = dev(c.K.view(np.int16) if c.dtype == "bf16" else c.K, kv_dtype)
+    V = dev(c.V.view(np.int16) if c.dtype == "bf16" else c.V, kv_dtype)
+    return hs2.KVCache(K=K, V=V, N=c.N, dtype=c.dtype, k_scale=dev(c.k_scale), v_scale=dev(c.v_scale),
+                       page_size=c.page_size, page_table=dev(c.page_table))
+
+
+def cache_to_numpy(cache):
+    """The binding's KVCache contents back as numpy code arrays (uint16 for bf16, uint8 for fp8)."""
+    if cache.dtype == "bf16":
+        return cache.K.view(torch.int16).cpu().numpy().view(np.uint16), cache.V.view(torch.int16).cpu().numpy().view(np.uint16)
+    return cache.K.view(torch.uint8).cpu().numpy(), cache.V.view(torch.uint8).cpu().numpy()

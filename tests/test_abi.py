@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert hs2.version() == "1.0"
+    assert hs2.version() == "1.1"
     for s in range(6):
         assert isinstance(hs2.status_string(s), str) and hs2.status_string(s)
 
@@ -147,3 +147,60 @@ def test_python_binding_refuses_tensors_on_two_devices():
         hs2.device_of("t", Q=on(0), K=on(1))
     with pytest.raises(ValueError, match="one CUDA device"):
         hs2.device_of("t", Q=on(0), K=on(0), ws=on(1))
+
+
+def _desc(**kw):
+    base = dict(dtype=hs2.KV_BF16, page_size=0, num_pages=0, max_pages=0, K=FAKE, V=FAKE, page_table=None,
+                k_scale=None, v_scale=None)
+    base.update(kw)
+    return hs2.KvCacheDesc(**base)
+
+
+def test_cache_descriptor_workspace_and_rejections(L):
+    d = _dims(N=4096)
+    ws_bf16 = L.hs2_workspace_size_kv(ctypes.byref(d), ctypes.byref(_desc()))
+    assert ws_bf16 == hs2.workspace_size(d)           # a contiguous bf16 descriptor is the plain call
+    paged = _desc(page_size=16, num_pages=300, max_pages=256, page_table=FAKE)
+    fp8 = _desc(dtype=hs2.KV_FP8_E4M3, k_scale=FAKE, v_scale=FAKE)
+    for desc in (paged, fp8, _desc(dtype=hs2.KV_FP8_E4M3, page_size=64, num_pages=70, max_pages=64,
+                                   page_table=FAKE, k_scale=FAKE, v_scale=FAKE)):
+        assert L.hs2_workspace_size_kv(ctypes.byref(d), ctypes.byref(desc)) > 0
+    # 128-row query tiles: fp8 and paged caches take the warp-level MMA sweeps (another plan)
+    pre = _dims(Hq=32, Hkv=4, T=4096, N=131072, k=2048, W=128)
+    assert L.hs2_workspace_size_kv(ctypes.byref(pre), ctypes.byref(fp8)) == \
+        L.hs2_workspace_size_kv(ctypes.byref(pre), ctypes.byref(_desc(page_size=64, num_pages=2048, max_pages=2048,
+                                                                       page_table=FAKE)))
+    bad_shapes = [_desc(page_size=24, num_pages=300, max_pages=256, page_table=FAKE),   # not a power of two
+                  _desc(page_size=4, num_pages=2000, max_pages=1024, page_table=FAKE),  # below 8
+                  _desc(page_size=16, num_pages=300, max_pages=255, page_table=FAKE),   # table too short
+                  _desc(page_size=16, num_pages=0, max_pages=256, page_table=FAKE),
+                  _desc(dtype=7)]
+    for desc in bad_shapes:
+        assert L.hs2_workspace_size_kv(ctypes.byref(d), ctypes.byref(desc)) == 0
+    assert L.hs2_workspace_size_kv(ctypes.byref(d), None) == 0
+    n = hs2.workspace_size(d) * 4
+    def step(desc, dims=d, ws_bytes=n):
+        return L.hs2_step_kv(ctypes.byref(dims), FAKE, FAKE, ctypes.byref(desc), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                             FAKE, FAKE, ws_bytes, None)
+    assert step(bad_shapes[0]) == hs2.HS2_ERR_INVALID_ARG
+    assert step(_desc(page_size=16, num_pages=300, max_pages=256)) == hs2.HS2_ERR_INVALID_ARG   # no page table
+    assert step(_desc(dtype=hs2.KV_FP8_E4M3)) == hs2.HS2_ERR_INVALID_ARG                        # no scales
+    assert step(_desc(K=FAKE + 8)) == hs2.HS2_ERR_INVALID_ARG                                   # misaligned cache
+    assert step(_desc(), ws_bytes=16) == hs2.HS2_ERR_WORKSPACE
+    assert step(_desc(), dims=_dims(d=96)) == hs2.HS2_ERR_UNSUPPORTED
+    # the decode step takes one query per batch row
+    t2 = _dims(T=2)
+    assert L.hs2_decode_step(ctypes.byref(t2), ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                             FAKE, FAKE, FAKE, FAKE, FAKE, n, None) == hs2.HS2_ERR_INVALID_ARG
+    # the append needs the 256-byte status word
+    assert L.hs2_kv_append(ctypes.byref(d), ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE, 128, None) == \
+        hs2.HS2_ERR_WORKSPACE
+
+
+def test_parity_checker_rejects_nan():
+    # a non-finite kernel output must fail the comparison, not slip through it
+    with pytest.raises(AssertionError):
+        parity.assert_close_o(np.array([0.5, np.nan]), np.array([0.5, 0.25]), "nan")
+    with pytest.raises(AssertionError):
+        parity.assert_close_lse(np.array([1.0, np.nan]), np.array([1.0, 2.0]), "nan")
+    parity.assert_close_o(np.array([0.5, 0.251]), np.array([0.5, 0.25]), "close")

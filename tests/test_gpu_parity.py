@@ -91,16 +91,6 @@ def test_step_matches_oracle(case):
     compare_step(inp, res)
 
 
-@pytest.mark.parametrize("case", [c for c in CASES if c[5] == 1], ids=lambda c: f"fused{c}")
-def test_decode_fused_kernel_matches_oracle(case, monkeypatch):
-    # T = 1 runs the kernel chain by default; check the opt-in single-kernel step too
-    monkeypatch.setenv("HS2_FUSED_DECODE", "1")
-    B, Hq, Hkv, d, N, T, k, W = case
-    inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 1, needles=4)
-    res = run_step(inp)
-    compare_step(inp, res)
-
-
 def test_positions_before_the_window_and_first_token():
     # pos < W (empty pool), pos = 0 (one visible key), and arbitrary positions per batch row
     pos = np.array([[0, 3, 10, 700], [5, 64, 65, 999]], np.int32)
