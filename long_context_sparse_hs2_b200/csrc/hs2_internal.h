@@ -153,6 +153,30 @@ struct ScoreArgs {         // scores + histogram from kept logits, with the full
     unsigned* status;
 };
 
+struct TailArgs {           // the decode step after the sweep, one cluster per selection row (k_tail.cu)
+    const float* logits;   // [rows_kv][N][G] base-2 logits of the sweep
+    const float2* pf_ml;   // full-attention split partials [S1][rows_q]
+    const float* pf_acc;   // [S1][rows_q][D]
+    int S1;
+    const uint16_t* Qs;    // Q_sparse [B][Hq][T][D]
+    const void* K;         // the cache (contiguous or pool), bf16 or E4M3 codes
+    const void* V;
+    KvSrc kv;
+    const int32_t* pos;    // [B][T]
+    int B, Hq, Hkv, T, N, k, W;
+    int stages;            // gather ring depth (set by the launcher)
+    float scale_log2;
+    uint16_t* O_full;
+    float* LSE_full;
+    uint16_t* O_sparse;
+    float* LSE_sparse;
+    int32_t* idx;          // [rows_kv][k+W]
+    int32_t* cnt;          // [rows_kv]
+    unsigned long long* cand;  // [rows_kv][cand_cap] candidate composites of the threshold bucket
+    int64_t cand_cap;
+    unsigned* status;
+};
+
 struct TopkArgs {
     const uint32_t* keys;  // [rows][kstride]
     int64_t kstride;
@@ -202,7 +226,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 int num_sms();  // streaming multiprocessors of the current device (queried once per device)
 
-cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st);  // clears ws[0, bytes) (normal launch)
+cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st);  // clears ws[0, bytes) once the stream's previous kernel is done
 
 // New tokens into the cache (hs2_kv_append / hs2_decode_step).  pos_in[b*T + t] (+1 when advance)
 // is the token's position; with advance (T = 1) the position is also written to pos_out[b] and
@@ -234,6 +258,9 @@ cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st);
 cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st);
+// The decode tail as one cluster kernel; *launched = false (nothing launched, cudaSuccess) when
+// the shape does not fit its plan -- the caller then runs score_hist, topk_select, sparse_attn.
+cudaError_t launch_tail(const Plan& p, const TailArgs& a, cudaStream_t st, bool* launched);
 cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st);
 
 }  // namespace hs2

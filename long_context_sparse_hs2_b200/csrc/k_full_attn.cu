@@ -279,19 +279,26 @@ cudaError_t launch_score_sweep(const Plan& p, int splits, const CUtensorMap& tmK
     return cudaErrorInvalidValue;
 }
 
+// Clears the start of the workspace (status word, counters) for the call that launches it.  It is
+// launched with programmatic serialisation, so it is resident while the stream's previous kernel
+// drains; it writes only after that kernel has completed (pdl_wait -- and since every kernel of
+// this library waits for its predecessor before it ends, the whole previous call has completed),
+// and lets the call's next kernel launch only after its own writes (the trigger comes last), so
+// nothing of this call touches the workspace while the previous call might still use it.
 __global__ void __launch_bounds__(256) init_kernel(uint4* p, int64_t n) {
-    pdl_trigger();
+    pdl_wait();
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         p[i] = make_uint4(0, 0, 0, 0);
+    pdl_trigger();
 }
 
 cudaError_t launch_init(void* ws, size_t bytes, cudaStream_t st) {
     const int64_t n = static_cast<int64_t>(bytes / 16);
     const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(8 * num_sms(), std::max<int64_t>(1, (n + 255) / 256)));
-    init_kernel<<<blocks, 256, 0, st>>>(static_cast<uint4*>(ws), n);
+    const cudaError_t e = launch_pdl(init_kernel, dim3(blocks), dim3(256), 0, st, static_cast<uint4*>(ws), n);
     trace_mark("init", st);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st) {

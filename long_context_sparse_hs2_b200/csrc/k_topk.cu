@@ -57,135 +57,6 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(const TopkArgs a) {
                              &s_last);
 }
 
-// ====================================================================== exact threshold among candidates
-
-namespace {
-
-struct SmemSource {
-    const unsigned long long* c;
-    int n;
-    __device__ int size() const { return n; }
-    __device__ bool get(int i, unsigned long long& v) const { v = c[i]; return true; }
-};
-struct GlobalSource {
-    const unsigned long long* c;
-    int n;
-    __device__ int size() const { return n; }
-    __device__ bool get(int i, unsigned long long& v) const { v = __ldcg(c + i); return true; }
-};
-struct KeyScanSource {  // overflow path: every pool key of the row whose bucket is b1
-    const uint32_t* keys;
-    int n, b1;
-    __device__ int size() const { return n; }
-    __device__ bool get(int i, unsigned long long& v) const {
-        const uint32_t k = __ldcg(keys + i);
-        v = composite(k, i);
-        return score_bin(k) == b1;
-    }
-};
-
-// The composite T such that exactly `need` source elements are >= T (8-bit radix digits,
-// most significant first; stops as soon as the remaining digits are free).
-template <class Src>
-__device__ unsigned long long radix_threshold(const Src& src, unsigned need, unsigned* h, unsigned* s_small) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // Bits every element shares need no pass: start at the highest digit where they differ.
-    __shared__ unsigned long long s_and[32], s_or[32];
-    unsigned long long all_and = ~0ull, any_or = 0ull;
-    for (int i = threadIdx.x; i < src.size(); i += blockDim.x) {
-        unsigned long long c;
-        if (src.get(i, c)) {
-            all_and &= c;
-            any_or |= c;
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        all_and &= __shfl_xor_sync(0xffffffffu, all_and, o);
-        any_or |= __shfl_xor_sync(0xffffffffu, any_or, o);
-    }
-    if (lane == 0) {
-        s_and[warp] = all_and;
-        s_or[warp] = any_or;
-    }
-    __syncthreads();
-    all_and = ~0ull;
-    any_or = 0ull;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
-        all_and &= s_and[w];
-        any_or |= s_or[w];
-    }
-    __syncthreads();
-    const unsigned long long differ = all_and ^ any_or;
-    if (differ == 0ull) return all_and;  // a single element (composites are distinct)
-    const int top = 63 - __clzll(static_cast<long long>(differ));
-    const int first_shift = (top / 8) * 8;
-    unsigned long long prefix = first_shift >= 56 ? 0ull : (all_and & (~0ull << (first_shift + 8)));
-    for (int shift = first_shift; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0u;
-        if (threadIdx.x == 0) s_small[0] = s_small[1] = 0u;
-        __syncthreads();
-        const unsigned long long mask_hi = (shift == 56) ? 0ull : (~0ull << (shift + 8));
-        const int n = src.size();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            unsigned long long c;
-            if (src.get(i, c) && (c & mask_hi) == (prefix & mask_hi))
-                atomicAdd(&h[static_cast<int>((c >> shift) & 255ull)], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            // lane covers digits 255-8*lane down to 248-8*lane (best first)
-            unsigned cnts[8], sum = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                cnts[i] = h[255 - 8 * lane - i];
-                sum += cnts[i];
-            }
-            unsigned incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const unsigned excl = incl - sum;
-            if (excl < need && need <= incl) {
-                unsigned cum = excl;
-                for (int i = 0; i < 8; ++i) {
-                    if (cum + cnts[i] >= need) {
-                        s_small[0] = 255 - 8 * lane - i;
-                        s_small[1] = cum;
-                        break;
-                    }
-                    cum += cnts[i];
-                }
-            }
-        }
-        __syncthreads();
-        const unsigned d = s_small[0];
-        need -= s_small[1];
-        prefix |= static_cast<unsigned long long>(d) << shift;
-        const bool done = (h[d] == need);
-        __syncthreads();
-        if (done) break;
-    }
-    return prefix;
-}
-
-// Writes the source elements >= thr; never more than `need` slots whatever the inputs.
-template <class Src>
-__device__ void emit_at_least(const Src& src, unsigned long long thr, unsigned need, int32_t* out, int* s_count) {
-    const int n = src.size();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        unsigned long long c;
-        if (src.get(i, c) && c >= thr) {
-            const int slot = atomicAdd(s_count, 1);
-            if (slot < static_cast<int>(need)) out[slot] = composite_index(c);
-        }
-    }
-}
-
-}  // namespace
-
 // ====================================================================== select: emit, then exact threshold
 
 __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
@@ -380,42 +251,6 @@ __device__ __forceinline__ void emit_bucket_range(const uint32_t* keys, int P, i
                 if (oc < kSmemCand) s_cand[oc] = composite(kk[e], j + e);
                 ++oc;
             }
-        }
-    }
-}
-
-// After a histogram in sh: for each of the two counts c[0], c[1] (>= 1), the smallest bucket b
-// whose cumulative count (buckets 0 .. b) reaches c, and the count below it, into
-// s_bin[i] / s_below[i] (bucket kHistBins - 1 and the count below it if c exceeds the total).
-// Call from all threads (NT of them).
-template <int NT>
-__device__ __forceinline__ void buckets_at_counts(const unsigned* sh, const unsigned (&c)[2], unsigned* s_warp,
-                                                  int* s_bin, int* s_below) {
-    constexpr int PER = kHistBins / NT;
-    const int tid = threadIdx.x;
-    unsigned vals[PER], sum = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        vals[i] = sh[tid * PER + i];
-        sum += vals[i];
-    }
-    const unsigned excl = block_exclusive_scan(sum, s_warp);
-    const bool last_thread = tid == NT - 1;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        if (excl < c[k] && c[k] <= excl + sum) {
-            unsigned cum = excl;
-            for (int i = 0; i < PER; ++i) {
-                if (cum + vals[i] >= c[k]) {
-                    s_bin[k] = tid * PER + i;
-                    s_below[k] = static_cast<int>(cum);
-                    break;
-                }
-                cum += vals[i];
-            }
-        } else if (last_thread && c[k] > excl + sum) {  // beyond the total
-            s_bin[k] = kHistBins - 1;
-            s_below[k] = static_cast<int>(excl + sum - vals[PER - 1]);
         }
     }
 }

@@ -223,3 +223,26 @@ def test_repeated_calls_reuse_workspace():
     for h in range(2):
         np.testing.assert_array_equal(np.sort(a["idx"][0, h, 0]), np.sort(b["idx"][0, h, 0]))
     compare_step(inp, b)
+
+
+TAIL_CASES = [c for c in CASES if c[5] * (c[1] // c[2]) <= 16]
+
+
+@pytest.mark.parametrize("cluster", ["1", "0"], ids=["cluster_tail", "kernel_chain"])
+@pytest.mark.parametrize("case", TAIL_CASES, ids=[str(c) for c in TAIL_CASES])
+def test_decode_tail_paths_match_oracle(case, cluster, monkeypatch):
+    # decode shapes run the selection and the sparse layer in one cluster kernel; the kernel
+    # chain (score_hist -> topk_select -> sparse_attn) stays for shapes the cluster plan does not
+    # fit (a million-token pool) and is checked here too (HS2_CLUSTER_TAIL=0)
+    monkeypatch.setenv("HS2_CLUSTER_TAIL", cluster)
+    B, Hq, Hkv, d, N, T, k, W = case
+    inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 7, needles=4)
+    hs2.trace_enable(True)
+    res = run_step(inp)
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    if cluster == "1":
+        assert "select_sparse_cluster" in kernels and "topk_select" not in kernels, kernels
+    else:
+        assert "select_sparse_cluster" not in kernels and "topk_select" in kernels, kernels
+    compare_step(inp, res)
