@@ -396,17 +396,31 @@ def run_gpu(w, kv_dtype, page_size, steps, warmup, e2e_steps, local_rank, dist):
     ms_e2e, h2d, d2h = None, 0, 0
     if e2e_steps > 0:
         # end to end through the public API with host buffers (pinned), copies inside the timed region
-        host_in = {n: t.cpu().pin_memory() for n, t in (("Qf", Qf), ("Qs", Qs), ("K", K), ("V", V), ("pos", pos))}
+        src = {"Qf": Qf, "Qs": Qs, "pos": pos}
+        if cache is None:
+            src.update(K=K, V=V)
+        else:
+            src.update({"cache_" + n: t for n, t in cache.tensors().items()})
+        host_in = {n: t.cpu().pin_memory() for n, t in src.items()}
         dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
         host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in out.as_dict().items()}
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        dev_cache = None
+        if cache is not None:
+            dev_cache = hs2.KVCache(K=dev_in["cache_K"], V=dev_in["cache_V"], N=cache.N, dtype=cache.dtype,
+                                    k_scale=dev_in.get("cache_k_scale"), v_scale=dev_in.get("cache_v_scale"),
+                                    page_size=cache.page_size, page_table=dev_in.get("cache_page_table"))
 
         def e2e_step():
             for n in dev_in:
                 dev_in[n].copy_(host_in[n], non_blocking=True)
-            hs2.step(dev_in["Qf"], dev_in["Qs"], dev_in["K"], dev_in["V"], dev_in["pos"], k=w.k, W=w.W, out=out,
-                     ws=ws, stream=stream)
+            if dev_cache is None:
+                hs2.step(dev_in["Qf"], dev_in["Qs"], dev_in["K"], dev_in["V"], dev_in["pos"], k=w.k, W=w.W, out=out,
+                         ws=ws, stream=stream)
+            else:
+                hs2.step_kv(dev_in["Qf"], dev_in["Qs"], dev_cache, dev_in["pos"], k=w.k, W=w.W, out=out, ws=ws,
+                            stream=stream)
             for n, t in out.as_dict().items():
                 host_out[n].copy_(t, non_blocking=True)
 
@@ -505,6 +519,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "fp8_e4m3"],
+                    help="how the headline workload's cache is stored")
+    ap.add_argument("--page-size", type=int, default=0, help="paged cache for the headline workload (0: contiguous)")
     ap.add_argument("--workloads", default=",".join(EXTRA_WORKLOADS),
                     help="comma-separated extra workloads timed after the headline one (one GPU), or 'none'")
     ap.add_argument("--extra-steps", type=int, default=20)
@@ -523,8 +540,8 @@ def main():
            "W": w.W, "global_batch": w.B * w.T * max(world, args.gpus), "seq_len": w.N,
            "parallelism": f"replicas x{max(world, args.gpus)}",
            "l2": (("flush: a %d MiB buffer is written between timed steps (K and V, %.1f MiB, fit in the 126 MB L2)"
-                   % (L2_FLUSH_BYTES >> 20, kv_bytes(w) / 2**20)) if kv_fits_l2(w) else
-                  "no flush: K and V (%d MiB) exceed the 126 MB L2" % (kv_bytes(w) >> 20))}
+                   % (L2_FLUSH_BYTES >> 20, kv_bytes(w, args.kv_dtype) / 2**20)) if kv_fits_l2(w, args.kv_dtype) else
+                  "no flush: K and V (%d MiB) exceed the 126 MB L2" % (kv_bytes(w, args.kv_dtype) >> 20))}
 
     if args.impl == "reference":
         if rank != 0:
@@ -549,7 +566,7 @@ def main():
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
     try:
-        r = run_gpu(w, "bf16", 0, args.steps, args.warmup, args.e2e_steps, local_rank, dist)
+        r = run_gpu(w, args.kv_dtype, args.page_size, args.steps, args.warmup, args.e2e_steps, local_rank, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
@@ -560,20 +577,23 @@ def main():
     n = max(world, 1)
     step_s = r["ms"] / 1000.0 / args.steps
     qps = replica_throughput(n, w.B * w.T, args.steps, r["ms"])
-    e2e_step_s = r["ms_e2e"] / 1000.0 / args.e2e_steps
     kern = kernel_table(r, args.steps)
     line = {
         "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_s * 1000.0, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q/K/V, needles, AR(1) drift)",
-        "config": cfg,
-        "hbm": hbm_block(w, "bf16", step_s, peaks),
-        "roofline": roofline(w, "bf16", kern, peaks, peak_src, w.name),
+        "vs_baseline": None, "dtype": "bf16" if args.kv_dtype == "bf16" else "bf16 queries, fp8 e4m3 KV cache",
+        "data": "synthetic (seeded N(0,1) Q/K/V, needles, AR(1) drift)",
+        "config": dict(cfg, kv_cache=args.kv_dtype + (f", paged ({args.page_size}-token pages)" if args.page_size
+                                                      else "")),
+        "hbm": hbm_block(w, args.kv_dtype, step_s, peaks),
+        "roofline": roofline(w, args.kv_dtype, kern, peaks, peak_src, w.name if args.kv_dtype == "bf16" and
+                             not args.page_size else None),
         "kernels": kern,
         "traced_ms_per_step": r["ms_traced"] / args.steps,
-        "e2e": {"value": replica_throughput(n, w.B * w.T, args.e2e_steps, r["ms_e2e"]), "unit": "queries/s",
-                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_step_s * 1000.0,
-                "steps": args.e2e_steps},
+        "e2e": ({"value": replica_throughput(n, w.B * w.T, args.e2e_steps, r["ms_e2e"]), "unit": "queries/s",
+                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                 "ms_per_step": r["ms_e2e"] / args.e2e_steps, "steps": args.e2e_steps}
+                if args.e2e_steps > 0 else None),
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }

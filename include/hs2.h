@@ -265,6 +265,15 @@ HS2_API hs2_status hs2_decode_step(const hs2_dims* dims, const hs2_kv_cache* cac
  * HS2_DEV_CAND_OVERFLOW is set, else HS2_OK. */
 HS2_API hs2_status hs2_read_device_status(const void* ws, void* stream, uint32_t* bits);
 
+/* Failure-detection self-test (not from the pages; a property of this library).  Every
+ * pipeline wait inside the kernels is bounded (2 s): when the bound runs out the kernel sets
+ * HS2_DEV_TIMEOUT in the status word and returns, so a stalled pipeline leaves an error instead
+ * of a hung GPU.  This call runs that same bounded wait, with the bound limit_ns (1 us .. 2 s), on
+ * a barrier that nothing ever arrives on, on `stream`.  Afterwards hs2_read_device_status(ws)
+ * returns HS2_ERR_DEVICE with exactly HS2_DEV_TIMEOUT set, after about limit_ns; the device stays
+ * usable.  ws: at least 256 bytes (the status word), 256-byte aligned. */
+HS2_API hs2_status hs2_selftest_wait_bound(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream);
+
 /* Static, human-readable name of a status code. */
 HS2_API const char* hs2_status_string(hs2_status status);
 

@@ -80,15 +80,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait until the phase with the given parity has completed, for at most kWaitLimitNs.
-// Returns false (and flags HS2_DEV_TIMEOUT) if the bound ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status) {
+// Wait until the phase with the given parity has completed, for at most limit_ns (kWaitLimitNs,
+// 2 s, unless a shorter bound is given).  Returns false (and flags HS2_DEV_TIMEOUT) if the bound
+// ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             pdl_wait();  // the status word is cleared by the call's first kernel
             set_status(status, HS2_DEV_TIMEOUT);
             return false;
@@ -99,43 +101,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 // Makes this thread's ordinary shared-memory stores visible to the async proxy (TMA, tensor
 // core) before a following barrier arrive.
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// ------------------------------------------------------------------ inter-CTA barrier (co-resident CTAs only)
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Barrier among the CTAs that share `ctr` (a counter cleared before the launch): each CTA adds
-// one and waits until the counter reaches `target` (= the number of barriers passed so far
-// times the number of participating CTAs).  Only for CTAs guaranteed to be co-resident
-// (cooperative launch).  The wait is bounded by kWaitLimitNs; on expiry it flags
-// HS2_DEV_TIMEOUT and returns false.  Writes made before the barrier are visible after it.
-__device__ __forceinline__ bool cta_barrier(unsigned* ctr, unsigned target, unsigned* status, int* s_flag) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        // release: this CTA's earlier writes are visible before the count; no round trip
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
-        int ok = 1;
-        if (ld_acquire(ctr) < target) {
-            const uint64_t t0 = global_ns();
-            while (ld_acquire(ctr) < target) {
-                if (global_ns() - t0 > kWaitLimitNs) {
-                    set_status(status, HS2_DEV_TIMEOUT);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(32);
-            }
-        }
-        __threadfence();  // acquire side: the other CTAs' writes are visible to the whole CTA
-        *s_flag = ok;
-    }
-    __syncthreads();
-    return *s_flag != 0;
-}
 
 // ------------------------------------------------------------------ L2 cache policies
 

@@ -34,7 +34,7 @@ ENTRY_POINTS = ("hs2_workspace_size", "hs2_full_attn", "hs2_select", "hs2_sparse
                 "hs2_read_device_status", "hs2_status_string", "hs2_trace_enable", "hs2_trace_collect",
                 "hs2_launch_count", "hs2_version", "hs2_sparse_attn_static", "hs2_workspace_size_kv",
                 "hs2_full_attn_kv", "hs2_select_kv", "hs2_sparse_attn_kv", "hs2_step_kv", "hs2_kv_append",
-                "hs2_decode_step")
+                "hs2_decode_step", "hs2_selftest_wait_bound")
 STATIC_SCRATCH_BYTES = 4 << 20  # HS2_STATIC_SCRATCH_BYTES
 
 
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
     for f in ("hs2_full_attn_kv", "hs2_select_kv", "hs2_sparse_attn_kv", "hs2_step_kv", "hs2_kv_append",
               "hs2_decode_step"):
         getattr(L, f).restype = ctypes.c_int
+    L.hs2_selftest_wait_bound.argtypes = [vp, sz, ctypes.c_uint64, vp]
+    L.hs2_selftest_wait_bound.restype = ctypes.c_int
     L.hs2_read_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.hs2_status_string.argtypes = [ctypes.c_int]
     L.hs2_status_string.restype = ctypes.c_char_p
@@ -516,6 +518,13 @@ def decode_step(Q_full, Q_sparse, cache: KVCache, K_new, V_new, pos, *, k: int, 
                                      _p(out.LSE_sparse), _p(out.idx), _p(out.cnt), _p(ws), ws.numel(),
                                      _stream(stream, dev)), "hs2_decode_step")
     return out
+
+
+def selftest_wait_bound(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """hs2_selftest_wait_bound: run a bounded device wait that runs out (sets DEV_TIMEOUT in ws)."""
+    with torch.cuda.device(ws.device):
+        _check(lib().hs2_selftest_wait_bound(_p(ws), ws.numel(), int(limit_ns), _stream(stream, ws.device)),
+               "hs2_selftest_wait_bound")
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:

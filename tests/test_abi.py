@@ -204,3 +204,10 @@ def test_parity_checker_rejects_nan():
     with pytest.raises(AssertionError):
         parity.assert_close_lse(np.array([1.0, np.nan]), np.array([1.0, 2.0]), "nan")
     parity.assert_close_o(np.array([0.5, 0.251]), np.array([0.5, 0.25]), "close")
+
+
+def test_wait_bound_selftest_argument_checks(L):
+    assert L.hs2_selftest_wait_bound(None, 256, 10_000, None) == hs2.HS2_ERR_WORKSPACE
+    assert L.hs2_selftest_wait_bound(FAKE, 128, 10_000, None) == hs2.HS2_ERR_WORKSPACE
+    assert L.hs2_selftest_wait_bound(FAKE, 256, 10, None) == hs2.HS2_ERR_INVALID_ARG            # below 1 us
+    assert L.hs2_selftest_wait_bound(FAKE, 256, 3_000_000_000, None) == hs2.HS2_ERR_INVALID_ARG  # above 2 s

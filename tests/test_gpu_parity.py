@@ -246,3 +246,17 @@ def test_decode_tail_paths_match_oracle(case, cluster, monkeypatch):
     else:
         assert "select_sparse_cluster" not in kernels and "topk_select" in kernels, kernels
     compare_step(inp, res)
+
+
+def test_bounded_wait_runs_out_and_the_device_stays_usable():
+    # a pipeline wait that nothing completes gives up after its bound, sets DEV_TIMEOUT and lets
+    # the kernel return; the next call on the same device works
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    hs2.selftest_wait_bound(ws, 2_000_000)  # 2 ms
+    e1.record()
+    assert hs2.read_device_status(ws) == hs2.DEV_TIMEOUT
+    assert 2.0 <= e0.elapsed_time(e1) < 200.0
+    inp = make_inputs(1, 8, 1, 128, 1000, 1, 37, 16, seed=9, needles=2)
+    compare_step(inp, run_step(inp))
