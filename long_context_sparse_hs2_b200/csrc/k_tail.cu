@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kTailThreads, 1) tail_kernel(const TailArgs a)
             const int ja = j0 + s * kStageKeys, jb = min(j1, ja + kStageKeys);
             const int lead = static_cast<int>((reinterpret_cast<uintptr_t>(lrow + static_cast<int64_t>(ja) * G * 4) & 15) / 4);
             const float* st = s_stage + (s & 1) * (kTailStageBytes / 4) + lead;
-            constexpr int U = 4;  // keys per thread in flight: independent chains hide the latencies
+            constexpr int U = 8;  // keys per thread in flight: independent chains hide the latencies
             for (int jb0 = ja + tid; jb0 < jb && ok; jb0 += U * kTailThreads) {
                 float v[U][G];
 #pragma unroll
