@@ -14,7 +14,7 @@ GPU (the step has no cross-GPU exchange); timing is the max over ranks.  Prints 
 line on rank 0.  ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
 
 On one GPU the same line also carries a ``workloads`` block: the other benchmark shapes
-(batched decode, chunked prefill, 1M-token decode at T = 1 and 16) and the headline shapes
+(tiny and batched decode, chunked prefill, 1M-token decode at T = 1 and 16) and the headline shapes
 with the cache stored as FP8 E4M3 or in a paged pool, each with its step time, queries/s,
 roofline, clocks and a bounded CPU-oracle baseline.
 """
@@ -44,6 +44,7 @@ L2_FLUSH_BYTES = 256 << 20
 # the headline shapes with the cache stored as FP8 E4M3 or in a paged pool.
 #   name -> (shape, cache dtype, page size)
 EXTRA_WORKLOADS = {
+    "tiny": ("tiny", "bf16", 0),
     "batched": ("batched", "bf16", 0),
     "prefill": ("prefill", "bf16", 0),
     "1m_t1": ("1m_t1", "bf16", 0),
@@ -451,13 +452,33 @@ def kernel_table(r, steps):
 def roofline(w, kv_dtype, kern, peaks, peak_src, name):
     """Roofline of the dominant kernel (the full-attention sweep) from its live CUDA-event time."""
     bm = byte_model(w, kv_dtype)
-    top = max((k for k in kern if k.startswith("full_attn") or k == "umma_attn"), key=lambda k: kern[k]["avg_us"],
-              default=None)
+    top = max((k for k in kern if k.startswith("full_attn") or k in ("umma_attn", "decode_fused")),
+              key=lambda k: kern[k]["avg_us"], default=None)
     if top is None:
         return None
     secs = kern[top]["avg_us"] * 1e-6
-    if top == "umma_attn":
-        # many query rows per kv head on the tcgen05 tensor cores: the sweep is a dense contraction
+    if top == "decode_fused":
+        # the whole decode step in one launch: K and V once, then the gathered selection rows
+        alg = bm["kv_once"] + bm["gathered"]
+        achieved = alg / secs / 1e9
+        return {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((name, top)),
+                "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "algorithmic_bytes_per_launch": alg}
+    # the tcgen05 sweep is a dense contraction; it is tensor-bound when its FLOPs take longer at
+    # the measured GEMM peak than its K/V bytes at the measured copy bandwidth (chunked prefill),
+    # HBM-bound otherwise (16 decode queries: 128 FLOPs per byte, below the ridge)
+    tensor_bound = top == "umma_attn" and (flop_model(w) / (peaks["bf16_tflops"] * 1e12) >
+                                           bm["kv_once"] / (peaks["hbm_gbs"] * 1e9))
+    if top == "umma_attn" and not tensor_bound:
+        achieved = bm["kv_once"] / secs / 1e9
+        flops = flop_model(w) / secs / 1e12
+        return {"bound": "hbm", "kernel": top, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((name, top)),
+                "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "algorithmic_bytes_per_launch": bm["kv_once"],
+                "tensor": {"achieved_tflops": flops, "frac_of_burst": flops / peaks["bf16_tflops"]}}
+    if tensor_bound:
         achieved = flop_model(w) / secs / 1e12
         return {"bound": "tensor", "kernel": top, "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,

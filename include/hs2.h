@@ -135,8 +135,11 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, c
  * chunked prefill, multi-query decode) the full-attention and score sweeps run on the tcgen05
  * tensor cores.  Two environment variables change the execution plan (results are the same up
  * to rounding order; the workspace size depends on them, so query hs2_workspace_size under the
- * same environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles.  The plan,
- * and so the workspace size, also follows the current device's SM count. */
+ * same environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles, and
+ * HS2_CLUSTER_TAIL=1 / 0 forces the decode tail after the sweep (T*G <= 16) onto one
+ * thread-block cluster per selection row / onto the three-kernel chain (by default each shape
+ * takes the one measured faster for it).  The plan, and so the workspace size, also follows the
+ * current device's SM count. */
 HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
                     const void* K, const void* V, const int32_t* pos,
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,

@@ -151,24 +151,16 @@ __device__ __forceinline__ void block_combine_row(const float2* __restrict__ par
     __syncthreads();
 }
 
-// The whole CTA merges the split partials of nh rows at once (the G query heads of one
-// selection row: rows row0 + g * stride).  Warps first turn each row's (m, l) into per-split
-// weights (s_w[g * S + s]); then every thread owns float4 columns (row, 4 dims) and sums its
-// splits with up to U loads in flight.  s_w: nh * S floats, s_ml: nh float2.  Call from all
-// threads (contains barriers).
+// Merge, for float4 columns col0, col0 + cstep, ... of nh rows (rows row0 + g * stride, D/4
+// columns each), the S split partials with the per-split weights s_w[g * S + s] and (M, L)
+// s_ml[g] already computed; writes bf16 O and (with a row's first column) the natural-log LSE.
+// Up to U loads in flight per column.  No barriers.
 template <int D, int U = 32>
-__device__ __forceinline__ void block_combine_rows(const float2* __restrict__ part_ml,
-                                                   const float* __restrict__ part_acc, int S, int64_t rows,
-                                                   int64_t row0, int64_t stride, int nh, float* s_w, float2* s_ml,
-                                                   uint16_t* O, float* LSE) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int g = warp; g < nh; g += nw) {
-        const float2 ML = warp_row_weights(part_ml, S, rows, row0 + g * stride, s_w + g * S);
-        if (lane == 0) s_ml[g] = ML;
-    }
-    __syncthreads();
+__device__ __forceinline__ void combine_columns(const float* __restrict__ part_acc, int S, int64_t rows, int64_t row0,
+                                                int64_t stride, int nh, const float* s_w, const float2* s_ml,
+                                                uint16_t* O, float* LSE, int col0, int cstep) {
     constexpr int C4 = D / 4;  // float4 columns per row
-    for (int col = threadIdx.x; col < nh * C4; col += blockDim.x) {
+    for (int col = col0; col < nh * C4; col += cstep) {
         const int g = col / C4, c = col % C4;
         const int64_t row = row0 + g * stride;
         const float* src = part_acc + row * D + c * 4;
@@ -193,6 +185,25 @@ __device__ __forceinline__ void block_combine_rows(const float2* __restrict__ pa
             make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
         if (c == 0) LSE[row] = lse2_of(s_ml[g]) * kLn2;
     }
+}
+
+// The whole CTA merges the split partials of nh rows at once (the G query heads of one
+// selection row: rows row0 + g * stride).  Warps first turn each row's (m, l) into per-split
+// weights (s_w[g * S + s]); then every thread owns float4 columns (row, 4 dims) and sums its
+// splits with up to U loads in flight.  s_w: nh * S floats, s_ml: nh float2.  Call from all
+// threads (contains barriers).
+template <int D, int U = 32>
+__device__ __forceinline__ void block_combine_rows(const float2* __restrict__ part_ml,
+                                                   const float* __restrict__ part_acc, int S, int64_t rows,
+                                                   int64_t row0, int64_t stride, int nh, float* s_w, float2* s_ml,
+                                                   uint16_t* O, float* LSE) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int g = warp; g < nh; g += nw) {
+        const float2 ML = warp_row_weights(part_ml, S, rows, row0 + g * stride, s_w + g * S);
+        if (lane == 0) s_ml[g] = ML;
+    }
+    __syncthreads();
+    combine_columns<D, U>(part_acc, S, rows, row0, stride, nh, s_w, s_ml, O, LSE, threadIdx.x, blockDim.x);
     __syncthreads();
 }
 

@@ -136,8 +136,25 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     // kernel's combine CTA G * S1 weights in its histogram scratch
     if (static_cast<int64_t>(G) * P.S4 > 8192 || static_cast<int64_t>(G) * P.S1 > 4096) return false;
     P.cand_cap = std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
-    const int64_t sparse_slots = P.S4;
+    // one-launch decode step: one selection row per row block, kept logits, every candidate list
+    // able to hold a whole pool, a split's pool keys within the kernel's shared-memory key buffer
+    const char* want_fused = std::getenv("HS2_FUSED_DECODE");
+    const int64_t tiles64 = (static_cast<int64_t>(x.N) + kKeyTile - 1) / kKeyTile;
+    P.fused = x.T == 1 && P.RT == 1 && P.mat_logits && !P.umma && P.cand_cap >= x.N &&
+              ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap && !(want_fused && want_fused[0] == '0');
+    const int64_t sparse_slots = P.fused ? std::max<int64_t>(P.S4, P.S1) : P.S4;
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
+    // bracketed selection (tcgen05 score sweep, many rows, large pools): a 1/16 tile sample per
+    // row instead of every key, and candidate lists of max(4096, 3 k) (never more than N)
+    const char* want_bracket = std::getenv("HS2_PREFILL_BRACKET");
+    P.bracketed = P.umma && rows_kv >= int64_t(kRowsPerCtaTopkPerSM) * sms && x.N >= kBracketMinPool &&
+                  4 * P.SS <= kMaxSegments && !(want_bracket && want_bracket[0] == '0');
+    P.sstride = ((static_cast<int64_t>(x.N) + 128 * kSampleTileStride - 1) / (128 * kSampleTileStride)) * 128;
+    P.bcap = std::min<int64_t>(x.N, std::max<int64_t>(4096, 3 * static_cast<int64_t>(x.k)));
+    // the filtering sweep's epilogue warps (four per split) each fill their own segment of a
+    // row's list: no atomics, and the keys of a tile are spread evenly over the four
+    P.nseg = 4 * P.SS;
+    P.seg_cap = static_cast<int>(P.bcap / P.nseg);
     // multi-CTA top-k: one chunk per CTA while that is a few waves; with many chunks in all
     // (1M keys x 64 rows) each CTA takes several, so launch and completion costs amortise
     const int64_t nchunks = (static_cast<int64_t>(x.N) + kTopkChunk - 1) / kTopkChunk;
@@ -149,14 +166,17 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     P.off_pos = off; off = align_up(off + size_t(x.B) * 4, 256);  // decode step: the positions it runs at
     P.off_meta = off; off = align_up(off + rows_kv * kMetaInts * 4, 256);
     P.meta_end = off;
-    P.off_hist = off; off = align_up(off + rows_kv * kHistBins * 4, 256);
+    // per-row global histograms: the multi-CTA top-k (few rows) and the kept-logits score kernel only
+    const bool need_hist = P.mat_logits || rows_kv < int64_t(kRowsPerCtaTopkPerSM) * sms;
+    P.off_hist = off; off = align_up(off + (need_hist ? rows_kv * kHistBins * 4 : 0), 256);
     P.zero_bytes = off;
     P.off_pf_ml = off; off = align_up(off + size_t(P.S1) * rows_q * 8, 256);
     P.off_pf_acc = off; off = align_up(off + size_t(P.S1) * rows_q * x.d * 4, 256);
     P.off_ps_ml = off; off = align_up(off + size_t(sparse_slots) * rows_q * 8, 256);
     P.off_ps_acc = off; off = align_up(off + size_t(sparse_slots) * rows_q * x.d * 4, 256);
-    P.off_keys = off; off = align_up(off + size_t(rows_kv) * P.kstride * 4, 256);
-    P.off_cand = off; off = align_up(off + size_t(rows_kv) * P.cand_cap * 8, 256);
+    P.off_keys = off; off = align_up(off + size_t(rows_kv) * (P.bracketed ? P.sstride : P.kstride) * 4, 256);
+    P.off_cand = off; off = align_up(off + size_t(rows_kv) * (P.bracketed ? P.bcap : P.cand_cap) * 8, 256);
+    P.off_segcnt = off; off = align_up(off + (P.bracketed ? size_t(rows_kv) * P.nseg * 4 : 0), 256);
     P.off_logits = off;
     if (P.mat_logits) off = align_up(off + size_t(rows_kv) * x.N * G * 4, 256);
     P.total = off;
@@ -314,6 +334,33 @@ hs2_status run_select_sweep(const Plan& p, const void* Qf, const KvView& kv, con
     a.kstride = p.kstride;
     a.k = p.k;
     a.S = p.S2;
+    if (p.bracketed) {
+        // sample -> bracket -> filtering sweep -> exact selection from the candidates
+        TopkArgs t = topk_args(p, pos, idx, cnt, w);
+        t.kstride = p.sstride;
+        t.cand_cap = p.bcap;
+        t.Q = static_cast<const uint16_t*>(Qf);
+        t.K = static_cast<const uint16_t*>(kv.K);
+        t.lse = LSE_full;
+        t.Hq = p.Hq; t.G = p.G; t.d = p.d;
+        t.scale_log2 = scale_log2(p);
+        t.segcnt = w.at<int>(p.off_segcnt);
+        t.nseg = p.nseg;
+        t.seg_cap = p.seg_cap;
+        a.score_mode = 1;
+        a.kstride = p.sstride;
+        HS2_TRY(launch_umma_score(p, tmK, a, st));
+        HS2_TRY(launch_topk_bracket(p, t, st));
+        a.score_mode = 2;
+        a.cand = w.at<unsigned long long>(p.off_cand);
+        a.cand_cap = p.bcap;
+        a.seg_cap = p.seg_cap;
+        a.segcnt = w.at<int>(p.off_segcnt);
+        a.meta = w.at<int>(p.off_meta);
+        HS2_TRY(launch_umma_score(p, tmK, a, st));
+        HS2_TRY(launch_topk_finalize(p, t, st));
+        return HS2_OK;
+    }
     if (p.umma)
         HS2_TRY(launch_umma_score(p, tmK, a, st));
     else
@@ -379,8 +426,11 @@ hs2_status run_tail(const Plan& p, const void* Qs, const KvView& kv, const int32
                     void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt, const Ws& w,
                     cudaStream_t st, bool* done) {
     *done = false;
+    // HS2_CLUSTER_TAIL=0: always the kernel chain; =1: the cluster kernel wherever it fits; unset:
+    // the cluster kernel where it measured faster (see launch_tail)
     const char* env = std::getenv("HS2_CLUSTER_TAIL");
     if (env && env[0] == '0') return HS2_OK;
+    const bool force = env && env[0] == '1';
     TailArgs t{};
     t.logits = w.at<float>(p.off_logits);
     t.pf_ml = w.at<float2>(p.off_pf_ml);
@@ -402,7 +452,38 @@ hs2_status run_tail(const Plan& p, const void* Qs, const KvView& kv, const int32
     t.cand = w.at<unsigned long long>(p.off_cand);
     t.cand_cap = p.cand_cap;
     t.status = w.at<unsigned>(p.off_status);
-    HS2_TRY(launch_tail(p, t, st, done));
+    HS2_TRY(launch_tail(p, t, st, force, done));
+    return HS2_OK;
+}
+
+// The one-launch decode step; *done = false when its grid does not fit on the device at once
+// (nothing launched).  The counters and histograms must have been cleared before.
+hs2_status run_fused(const Plan& p, const void* Qf, const void* Qs, const KvView& kv, const int32_t* pos,
+                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt,
+                     const Ws& w, cudaStream_t st, bool pdl, bool* done) {
+    *done = false;
+    CUtensorMap tmK, tmV;
+    if (!make_kv_map(&tmK, kv.K, p, kKeyTile) || !make_kv_map(&tmV, kv.V, p, kKeyTile)) return HS2_ERR_CUDA;
+    AttnArgs a = attn_args(p, Qf, pos, kv, w);
+    a.logits = w.at<float>(p.off_logits);
+    FusedArgs f{};
+    f.Qs = static_cast<const uint16_t*>(Qs);
+    f.K = kv.K;
+    f.V = kv.V;
+    f.k = p.k;
+    f.O_full = static_cast<uint16_t*>(O_full);
+    f.LSE_full = LSE_full;
+    f.O_sparse = static_cast<uint16_t*>(O_sparse);
+    f.LSE_sparse = LSE_sparse;
+    f.idx = idx;
+    f.cnt = cnt;
+    f.hist = w.at<unsigned>(p.off_hist);
+    f.meta = w.at<int>(p.off_meta);
+    f.cand = w.at<unsigned long long>(p.off_cand);
+    f.cand_cap = p.cand_cap;
+    f.ps_ml = w.at<float2>(p.off_ps_ml);
+    f.ps_acc = w.at<float>(p.off_ps_acc);
+    HS2_TRY(launch_decode_fused(p, tmK, tmV, a, f, st, pdl, done));
     return HS2_OK;
 }
 
@@ -410,6 +491,12 @@ hs2_status run_tail(const Plan& p, const void* Qs, const KvView& kv, const int32
 hs2_status run_step(const Plan& p, const void* Qf, const void* Qs, const KvView& kv, const int32_t* pos,
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt,
                     const Ws& w, cudaStream_t st, bool first_pdl) {
+    if (p.fused) {  // the caller cleared the counters and histograms (init over zero_bytes)
+        bool done = false;
+        const hs2_status s = run_fused(p, Qf, Qs, kv, pos, O_full, O_sparse, LSE_full, LSE_sparse, idx, cnt, w, st,
+                                       first_pdl, &done);
+        if (s != HS2_OK || done) return s;
+    }
     hs2_status s = run_full(p, Qf, kv, pos, O_full, LSE_full, w, p.mat_logits, !p.mat_logits, p.off_meta,
                             p.zero_bytes, st, first_pdl);
     if (s != HS2_OK) return s;
@@ -521,7 +608,9 @@ hs2_status step_impl(const Plan& p, const KvView& kv, const void* Q_full, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(launch_init(ws, 256, st));  // status word; the full sweep clears the rest
+    // status word (and, for the one-launch decode step, the counters and histograms; otherwise
+    // the full sweep clears those for the kernels after it)
+    HS2_TRY(launch_init(ws, p.fused ? p.zero_bytes : 256, st));
     return run_step(p, Q_full, Q_sparse, kv, pos, O_full, O_sparse, LSE_full, LSE_sparse, idx, cnt, w, st, true);
 }
 
@@ -671,7 +760,7 @@ hs2_status hs2_decode_step(const hs2_dims* dims, const hs2_kv_cache* cache, cons
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(launch_init(ws, 256, st));  // status word
+    HS2_TRY(launch_init(ws, p.fused ? p.zero_bytes : 256, st));  // status word (+ counters: see step_impl)
     // the new tokens go in and pos advances; the step then reads the positions from ws.  The full
     // sweep is an ordinary launch, so it starts after the append has completed and every kernel
     // after it sees the new tokens and positions.

@@ -28,9 +28,13 @@ constexpr int kMetaInts = 8;
 enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDef = 2, kMetaCand = 3, kMetaDone = 4, kMetaSelDone = 5,
                 kMetaSparseDone = 6, kMetaBarrier = 7 };  // kMetaDef/kMetaCand share one 8-byte word
 constexpr int kSmemCand = 4096;      // candidates the final select keeps in shared memory
+constexpr int kFusedKeyCap = 16384;  // pool keys per split of the one-launch decode step
 constexpr int kMaxKW = 1 << 22;      // largest supported k + W
 constexpr int kSparseMaxC4 = 4096;         // most selected keys one sparse-attention CTA takes
 constexpr int kRowsPerCtaTopkPerSM = 4;   // from 4 x (SMs) selection rows on, one top-k CTA per row
+constexpr int kSampleTileStride = 16;      // bracketed path: one 128-key tile in 16 is sampled
+constexpr int kBracketMinPool = 32768;     // bracketed path: only for caches of at least this many keys
+constexpr int kMaxSegments = 64;          // candidate-list segments per row on the bracketed path
 
 // How the kernels find a token's K/V row in the cache (see hs2_kv_cache in hs2.h).
 //   contiguous: row (b*Hkv + h)*N + j of [B][Hkv][N][d]
@@ -71,8 +75,16 @@ struct Plan {
     bool paged;         // the cache is a paged pool
     int page_size, max_pages, num_pages;
     int sms;            // streaming multiprocessors of the device the plan was made for
+    // Many rows on the tcgen05 score sweep with large pools: the sweep never stores every key.
+    // A pass over a 1/16 sample of the key tiles brackets each row's threshold bucket, and the
+    // full pass appends only the keys at or above it to the row's candidate list.
+    bool bracketed;
+    int nseg, seg_cap;  // bracketed: candidate-list segments per row (4 per score split) and their size
+    bool fused;         // decode (T = 1): the one-launch step (k_decode_fused.cu), where its grid fits
+    int64_t sstride;    // sample keys per row (a multiple of 128)
+    int64_t bcap;       // candidate-list capacity per row
     // workspace byte offsets
-    size_t off_status, off_pos, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand,
+    size_t off_status, off_pos, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand, off_segcnt,
         off_logits, zero_bytes, total;
 };
 
@@ -104,6 +116,18 @@ struct AttnArgs {
     uint32_t* keys;        // [rows_kv][kstride] order-preserving score keys (score sweep only)
     int64_t kstride;
     int k;
+    // tcgen05 score sweep: 0 stores every pool key's score key in keys; 1 scores every
+    // kSampleTileStride-th 128-key tile and stores them compactly in keys (the sample); 2 writes
+    // the composite (key, ~j) of every pool key whose bucket is at most the row's bracket
+    // (meta[row][kMetaBin]) to the candidate list cand[row] (row stride cand_cap): each epilogue
+    // warp of each split fills its own segment of seg_cap entries, and segcnt[row][segment]
+    // receives the segment's count (which may exceed seg_cap: the list then overflowed)
+    int score_mode;
+    unsigned long long* cand;
+    int64_t cand_cap;
+    int seg_cap;
+    int* segcnt;
+    int* meta;
     KvSrc kv;              // cache layout / dtype (TMA producer and scales)
     unsigned* status;
 };
@@ -153,6 +177,25 @@ struct ScoreArgs {         // scores + histogram from kept logits, with the full
     unsigned* status;
 };
 
+struct FusedArgs {          // the selection and sparse layer of the one-launch decode step
+    const uint16_t* Qs;    // Q_sparse [B][Hq][1][D]
+    const void* K;         // the cache (contiguous or pool), bf16 or E4M3 codes
+    const void* V;
+    int k;
+    uint16_t* O_full;      // [B][Hq][1][D]
+    float* LSE_full;       // [B][Hq][1]
+    uint16_t* O_sparse;
+    float* LSE_sparse;
+    int32_t* idx;          // [rows_kv][k+W]
+    int32_t* cnt;          // [rows_kv]
+    unsigned* hist;        // [rows_kv][kHistBins], cleared before the launch
+    int* meta;             // [rows_kv][kMetaInts], cleared before the launch
+    unsigned long long* cand;  // [rows_kv][cand_cap] threshold-bucket candidates (cand_cap >= N)
+    int64_t cand_cap;
+    float2* ps_ml;         // sparse split partials [S][rows_q]
+    float* ps_acc;         // [S][rows_q][D]
+};
+
 struct TailArgs {           // the decode step after the sweep, one cluster per selection row (k_tail.cu)
     const float* logits;   // [rows_kv][N][G] base-2 logits of the sweep
     const float2* pf_ml;   // full-attention split partials [S1][rows_q]
@@ -178,8 +221,16 @@ struct TailArgs {           // the decode step after the sweep, one cluster per 
 };
 
 struct TopkArgs {
-    const uint32_t* keys;  // [rows][kstride]
+    const uint32_t* keys;  // [rows][kstride] (the sample keys for the bracket kernel)
     int64_t kstride;
+    // the exact fallback of the bracketed path rescores a row from Q, K and LSE (contiguous bf16)
+    const uint16_t* Q;     // Q_full [B][Hq][T][d]
+    const uint16_t* K;     // [B][Hkv][N][d]
+    const float* lse;      // LSE_full [B][Hq][T]
+    int Hq, G, d;
+    float scale_log2;
+    const int* segcnt;     // bracketed path: candidates per segment [rows][nseg], seg_cap per segment
+    int nseg, seg_cap;
     const int32_t* pos;    // [B][T]
     int Hkv, T, N, k, W;
     int64_t rows;
@@ -258,9 +309,20 @@ cudaError_t launch_score_hist(const Plan& p, const ScoreArgs& a, cudaStream_t st
 cudaError_t launch_combine(int d, const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st);
 cudaError_t launch_topk_hist(const Plan& p, const TopkArgs& a, cudaStream_t st);
+// The bracketed path: per row, the sample's bucket bracket (into meta[row][kMetaBin]) ...
+cudaError_t launch_topk_bracket(const Plan& p, const TopkArgs& a, cudaStream_t st);
+// ... and, after the filtering sweep, the exact selection from the candidate list (an exact
+// rescoring of the row where the bracket did not hold).
+cudaError_t launch_topk_finalize(const Plan& p, const TopkArgs& a, cudaStream_t st);
 // The decode tail as one cluster kernel; *launched = false (nothing launched, cudaSuccess) when
-// the shape does not fit its plan -- the caller then runs score_hist, topk_select, sparse_attn.
-cudaError_t launch_tail(const Plan& p, const TailArgs& a, cudaStream_t st, bool* launched);
+// the shape does not fit its plan, or (unless force) when the kernel chain measured faster for
+// it -- the caller then runs score_hist, topk_select, sparse_attn.
+cudaError_t launch_tail(const Plan& p, const TailArgs& a, cudaStream_t st, bool force, bool* launched);
 cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st);
+// The one-launch decode step (T = 1): sweep, selection and sparse layer in one cooperative grid
+// of p.S1 x rows_kv CTAs.  *launched = false (nothing launched, cudaSuccess) when the grid does
+// not fit on the device at once; the caller then runs the kernel chain.
+cudaError_t launch_decode_fused(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
+                                const FusedArgs& f, cudaStream_t st, bool pdl, bool* launched);
 
 }  // namespace hs2

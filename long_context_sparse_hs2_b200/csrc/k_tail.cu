@@ -527,8 +527,10 @@ struct TailChoice {
 struct TailKey {
     const void* kern;
     int dev, rows, N, kw, W;
+    bool force;
     bool operator==(const TailKey& o) const {
-        return kern == o.kern && dev == o.dev && rows == o.rows && N == o.N && kw == o.kw && W == o.W;
+        return kern == o.kern && dev == o.dev && rows == o.rows && N == o.N && kw == o.kw && W == o.W &&
+               force == o.force;
     }
 };
 
@@ -538,7 +540,7 @@ std::vector<std::pair<TailKey, TailChoice>> g_tail_cache;
 // Cluster size: the largest C (16 at most, any integer) that keeps every row's cluster resident at once,
 // with each CTA's share of the pool and of the selection within its shared-memory plan.
 template <int D, int G, bool FP8, class Kern>
-cudaError_t choose_tail(const Plan& p, Kern kern, TailChoice* out) {
+cudaError_t choose_tail(const Plan& p, Kern kern, bool force, TailChoice* out) {
     using L = TailSmem<D, FP8>;
     const int64_t kw = static_cast<int64_t>(p.k) + p.W;
     const int64_t pool_max = std::max<int64_t>(0, p.N - p.W);
@@ -576,6 +578,11 @@ cudaError_t choose_tail(const Plan& p, Kern kern, TailChoice* out) {
         }
         if (static_cast<int64_t>(active) < p.rows_kv && C > 1) continue;  // not one wave: try smaller clusters
         if (active < 1) return cudaSuccess;                               // cannot run: keep the kernel chain
+        // Measured on B200: the cluster tail beats the kernel chain when its grid covers most SMs
+        // (batched decode, 32 rows x 4 CTAs: 0.1425 against 0.1459 ms) and loses slightly when it
+        // leaves them idle (long-context decode, 8 rows x 10 CTAs: 0.1306 against 0.1292 ms).
+        // Unless forced, it takes the shape only when rows x C >= 4/5 of the SMs.
+        if (!force && static_cast<int64_t>(C) * p.rows_kv * 5 < static_cast<int64_t>(p.sms) * 4) return cudaSuccess;
         *out = TailChoice{C, s, bytes};
         return cudaSuccess;
     }
@@ -583,14 +590,14 @@ cudaError_t choose_tail(const Plan& p, Kern kern, TailChoice* out) {
 }
 
 template <int D, int G, bool FP8>
-cudaError_t tail_variant(const Plan& p, const TailArgs& x, cudaStream_t st, bool* launched) {
+cudaError_t tail_variant(const Plan& p, const TailArgs& x, cudaStream_t st, bool force, bool* launched) {
     using L = TailSmem<D, FP8>;
     auto kern = tail_kernel<D, G, FP8>;
     const int64_t kw = static_cast<int64_t>(p.k) + p.W;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
     const TailKey key{reinterpret_cast<const void*>(kern), dev, static_cast<int>(p.rows_kv), p.N, static_cast<int>(kw),
-                      p.W};
+                      p.W, force};
     TailChoice ch{-1, 0, 0};
     {
         std::lock_guard<std::mutex> lock(g_tail_mutex);
@@ -599,7 +606,7 @@ cudaError_t tail_variant(const Plan& p, const TailArgs& x, cudaStream_t st, bool
     }
     if (ch.C < 0) {
         ch = TailChoice{0, 0, 0};
-        const cudaError_t e = choose_tail<D, G, FP8>(p, kern, &ch);
+        const cudaError_t e = choose_tail<D, G, FP8>(p, kern, force, &ch);
         if (e != cudaSuccess) return e;
         std::lock_guard<std::mutex> lock(g_tail_mutex);
         g_tail_cache.emplace_back(key, ch);
@@ -634,23 +641,25 @@ cudaError_t tail_variant(const Plan& p, const TailArgs& x, cudaStream_t st, bool
 }
 
 template <int D, bool FP8>
-cudaError_t tail_g(const Plan& p, const TailArgs& x, cudaStream_t st, bool* launched) {
+cudaError_t tail_g(const Plan& p, const TailArgs& x, cudaStream_t st, bool force, bool* launched) {
     switch (p.G) {
-        case 1: return tail_variant<D, 1, FP8>(p, x, st, launched);
-        case 2: return tail_variant<D, 2, FP8>(p, x, st, launched);
-        case 4: return tail_variant<D, 4, FP8>(p, x, st, launched);
-        case 8: return tail_variant<D, 8, FP8>(p, x, st, launched);
-        case 16: return tail_variant<D, 16, FP8>(p, x, st, launched);
+        case 1: return tail_variant<D, 1, FP8>(p, x, st, force, launched);
+        case 2: return tail_variant<D, 2, FP8>(p, x, st, force, launched);
+        case 4: return tail_variant<D, 4, FP8>(p, x, st, force, launched);
+        case 8: return tail_variant<D, 8, FP8>(p, x, st, force, launched);
+        case 16: return tail_variant<D, 16, FP8>(p, x, st, force, launched);
     }
     return cudaSuccess;
 }
 
 }  // namespace
 
-cudaError_t launch_tail(const Plan& p, const TailArgs& a, cudaStream_t st, bool* launched) {
+cudaError_t launch_tail(const Plan& p, const TailArgs& a, cudaStream_t st, bool force, bool* launched) {
     *launched = false;
-    if (p.d == 128) return p.fp8 ? tail_g<128, true>(p, a, st, launched) : tail_g<128, false>(p, a, st, launched);
-    if (p.d == 64) return p.fp8 ? tail_g<64, true>(p, a, st, launched) : tail_g<64, false>(p, a, st, launched);
+    if (p.d == 128)
+        return p.fp8 ? tail_g<128, true>(p, a, st, force, launched) : tail_g<128, false>(p, a, st, force, launched);
+    if (p.d == 64)
+        return p.fp8 ? tail_g<64, true>(p, a, st, force, launched) : tail_g<64, false>(p, a, st, force, launched);
     return cudaSuccess;
 }
 

@@ -373,6 +373,247 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkArgs a) {
     }
 }
 
+// ====================================================================== bracketed selection (unstored keys)
+//
+// With long pools and many rows (prefill) the keys are never stored.  The tcgen05 score sweep
+// first scores one 128-key tile in kSampleTileStride (keys compacted per row); topk_bracket
+// turns each row's sample into a bucket bracket b_hi -- the bucket of the sample key at rank
+// (expected rank of the keff-th best key) + margin; a second, filtering sweep writes every key
+// of bucket <= b_hi to the row's candidate list (each epilogue warp of the sweep fills its own
+// segment, so no atomics); topk_finalize radix-selects the exact top-keff among them.  A key of a bucket above b_hi scores strictly below every candidate, so the
+// result is exact whenever the list holds at least keff keys and nothing overflowed; where it
+// did not (an unlucky sample, heavy ties) topk_finalize rescores the row from Q, K and LSE on
+// the CUDA cores and selects exactly (flagged HS2_DEV_CAND_OVERFLOW, informational).
+
+__global__ void __launch_bounds__(256) topk_bracket_kernel(const TopkArgs a) {
+    __shared__ unsigned sh[kHistBins];
+    __shared__ unsigned s_warp[32];
+    __shared__ int s_bin[2], s_below[2];
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x;
+    pdl_trigger();
+    for (int i = tid; i < kHistBins; i += blockDim.x) sh[i] = 0u;
+    if (tid == 0) {
+        s_bin[0] = s_bin[1] = kHistBins - 1;
+        s_below[0] = s_below[1] = 0;
+    }
+    const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
+    int* meta = a.meta + row * kMetaInts;
+    pdl_wait();  // sample keys from the sampling sweep; the previous readers of meta are done
+    if (ri.keff == 0 || ri.keff == ri.P) {  // nothing to rank: the filter takes no key
+        if (tid == 0) meta[kMetaBin] = -1;
+        return;
+    }
+    constexpr int kSpan = kSampleTileStride * 128;  // pool keys per sample tile
+    const int nv = (ri.P + kSpan - 1) / kSpan;      // sample tiles (the last one may be short)
+    const int ns = 128 * (nv - 1) + min(128, ri.P - kSpan * (nv - 1));
+    const float r = static_cast<float>(ri.keff) * static_cast<float>(ns) / static_cast<float>(ri.P);
+    const float margin = 4.f * sqrtf(r) + 16.f;
+    if (ns < 256 || r + margin >= static_cast<float>(ns)) {  // too small a sample: every key is a candidate
+        if (tid == 0) meta[kMetaBin] = kHistBins - 1;
+        return;
+    }
+    __syncthreads();
+    const uint32_t* keys = a.keys + row * a.kstride;
+    for (int i = tid; i < nv * 128; i += blockDim.x) {
+        const int v = i >> 7, rr = i & 127;
+        if (rr < ri.P - kSpan * v) atomicAdd(&sh[score_bin(__ldcs(keys + i))], 1u);
+    }
+    __syncthreads();
+    const unsigned c = static_cast<unsigned>(r + margin) + 1u;
+    const unsigned cc[2] = {c, c};
+    buckets_at_counts<256>(sh, cc, s_warp, s_bin, s_below);
+    __syncthreads();
+    if (tid == 0) meta[kMetaBin] = s_bin[0];
+}
+
+namespace {
+
+// The selection key of pool key j for one row, recomputed on the CUDA cores: max over the G
+// heads of (q_g . k_j - u_g) scaled to base 2 (u_g = LSE_g sqrt(d), q in shared memory as fp32).
+struct Rescorer {
+    const uint16_t* K;  // this (b, kv head)'s keys [N][d]
+    const float* q;     // [G][d]
+    const float* u;     // [G]
+    int G, d;
+    float c2;
+    __device__ uint32_t key(int j) const {
+        const uint4* kr = reinterpret_cast<const uint4*>(K + static_cast<int64_t>(j) * d);
+        float best = -INFINITY;
+        bool nan = false;
+        for (int g = 0; g < G; ++g) {
+            const float* qg = q + g * d;
+            float x = 0.f;
+            for (int c = 0; c < d / 8; ++c) {
+                const uint4 w = __ldg(kr + c);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x = fmaf(qg[8 * c + 2 * e], __uint_as_float(ww[e] << 16), x);
+                    x = fmaf(qg[8 * c + 2 * e + 1], __uint_as_float(ww[e] & 0xFFFF0000u), x);
+                }
+            }
+            const float v = x - u[g];
+            nan |= v != v;
+            best = fmaxf(best, v);
+        }
+        return nan ? 0u : score_key(best * c2);  // NaN ranks below every score
+    }
+};
+
+struct SegmentSource {  // the candidates of a row's list segments (seg_start: nseg + 1 prefix offsets)
+    const unsigned long long* c;
+    const int* seg_start;
+    int nseg, seg_cap, n;
+    __device__ int size() const { return n; }
+    __device__ bool get(int i, unsigned long long& v) const {
+        int sg = 0;
+        while (sg + 1 < nseg && i >= seg_start[sg + 1]) ++sg;
+        v = __ldcg(c + sg * seg_cap + (i - seg_start[sg]));
+        return true;
+    }
+};
+
+struct RescoreSource {  // the pool keys of bucket b1, recomputed
+    Rescorer rs;
+    int n, b1;
+    __device__ int size() const { return n; }
+    __device__ bool get(int i, unsigned long long& v) const {
+        const uint32_t k = rs.key(i);
+        v = composite(k, i);
+        return score_bin(k) == b1;
+    }
+};
+
+}  // namespace
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_finalize_kernel(const TopkArgs a) {
+    __shared__ unsigned long long s_cand[kSmemCand];  // candidates; the fallback keeps Q here
+    __shared__ unsigned sh[kHistBins];
+    __shared__ unsigned h[256];
+    __shared__ unsigned s_small[2];
+    __shared__ unsigned s_warp[32];
+    __shared__ float s_u[16];
+    __shared__ int s_bin[2], s_below[2], s_ndef, s_ncand, s_count;
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x;
+    pdl_trigger();
+    if (tid == 0) {
+        s_ndef = s_ncand = s_count = 0;
+        s_bin[0] = s_bin[1] = kHistBins - 1;
+        s_below[0] = s_below[1] = 0;
+    }
+    const RowInfo ri = make_row_info(a.pos, row, a.Hkv, a.T, a.N, a.k, a.W);
+    const int kw = a.k + a.W;
+    int32_t* idx = a.idx + row * kw;
+    int32_t* out = idx + ri.wcnt;
+    pdl_wait();  // candidates from the filtering sweep
+    for (int i = tid; i < ri.wcnt; i += NT) idx[i] = ri.pos - ri.wcnt + 1 + i;
+    for (int i = ri.wcnt + ri.keff + tid; i < kw; i += NT) idx[i] = -1;
+    if (tid == 0) a.cnt[row] = ri.wcnt + ri.keff;
+    if (ri.keff == 0) return;
+    if (ri.keff == ri.P) {  // the whole pool is selected
+        for (int j = tid; j < ri.P; j += NT) out[j] = j;
+        return;
+    }
+    unsigned long long* gcand = a.cand + row * a.cand_cap;
+    // the candidates: nseg segments of the row's list, each filled by one epilogue warp
+    __shared__ int s_seg[kMaxSegments + 1];
+    __shared__ int s_over;
+    if (tid == 0) {
+        int total = 0, over = 0;
+        for (int sg = 0; sg < a.nseg; ++sg) {
+            const int c = __ldcg(a.segcnt + row * a.nseg + sg);
+            over |= c > a.seg_cap;
+            s_seg[sg] = total;
+            total += min(c, a.seg_cap);
+        }
+        s_seg[a.nseg] = total;
+        s_over = over;
+    }
+    __syncthreads();
+    const int n = s_seg[a.nseg];
+    if (!s_over && n >= ri.keff) {  // bracketed: the exact top-keff among the candidates
+        const unsigned need = static_cast<unsigned>(ri.keff);
+        if (n <= kSmemCand) {
+            for (int sg = 0; sg < a.nseg; ++sg) {
+                const int c = s_seg[sg + 1] - s_seg[sg];
+                for (int i = tid; i < c; i += NT) s_cand[s_seg[sg] + i] = __ldcg(gcand + sg * a.seg_cap + i);
+            }
+            __syncthreads();
+            const SmemSource src{s_cand, n};
+            emit_at_least(src, radix_threshold(src, need, h, s_small), need, out, &s_count);
+        } else {
+            const SegmentSource src{gcand, s_seg, a.nseg, a.seg_cap, n};
+            emit_at_least(src, radix_threshold(src, need, h, s_small), need, out, &s_count);
+        }
+        return;
+    }
+
+    // not bracketed: rescore the row (exact two-pass method on recomputed keys)
+    if (tid == 0) set_status(a.status, HS2_DEV_CAND_OVERFLOW);
+    const int t = static_cast<int>(row % a.T);
+    const int64_t bh = row / a.T;  // b * Hkv + kv head
+    const int b = static_cast<int>(bh / a.Hkv), hk = static_cast<int>(bh % a.Hkv);
+    float* s_q = reinterpret_cast<float*>(s_cand);  // G * d <= 2048 floats
+    const float sqrt_d = sqrtf(static_cast<float>(a.d));
+    for (int i = tid; i < a.G * a.d; i += NT) {
+        const int g = i / a.d, c = i % a.d;
+        const int64_t hq = static_cast<int64_t>(b) * a.Hq + hk * a.G + g;
+        s_q[i] = __uint_as_float(static_cast<uint32_t>(a.Q[(hq * a.T + t) * a.d + c]) << 16);
+    }
+    for (int g = tid; g < a.G; g += NT) s_u[g] = a.lse[(static_cast<int64_t>(b) * a.Hq + hk * a.G + g) * a.T + t] * sqrt_d;
+    for (int i = tid; i < kHistBins; i += NT) sh[i] = 0u;
+    __syncthreads();
+    const Rescorer rs{a.K + bh * a.N * a.d, s_q, s_u, a.G, a.d, a.scale_log2};
+    for (int j = tid; j < ri.P; j += NT) atomicAdd(&sh[score_bin(rs.key(j))], 1u);
+    __syncthreads();
+    {
+        const unsigned c[2] = {static_cast<unsigned>(ri.keff), static_cast<unsigned>(ri.keff)};
+        buckets_at_counts<NT>(sh, c, s_warp, s_bin, s_below);
+    }
+    __syncthreads();
+    const int b1 = s_bin[0], above = s_below[0];
+    if (above < 0 || above >= ri.keff) return;  // cannot happen for a consistent histogram
+    // better buckets go straight out; the threshold bucket's keys become the row's candidates
+    for (int j = tid; j < ri.P; j += NT) {
+        const uint32_t k = rs.key(j);
+        const int bin = score_bin(k);
+        if (bin < b1) {
+            const int slot = atomicAdd(&s_ndef, 1);
+            if (slot < above) out[slot] = j;
+        } else if (bin == b1) {
+            const int slot = atomicAdd(&s_ncand, 1);
+            if (slot < a.cand_cap) gcand[slot] = composite(k, j);
+        }
+    }
+    __syncthreads();
+    const unsigned need = static_cast<unsigned>(ri.keff - above);
+    const int ncand = s_ncand;
+    if (ncand <= a.cand_cap) {
+        const GlobalSource src{gcand, ncand};
+        emit_at_least(src, radix_threshold(src, need, h, s_small), need, out + above, &s_count);
+    } else {  // more ties in one bucket than the list holds: recompute them on every pass
+        const RescoreSource src{rs, ri.P, b1};
+        emit_at_least(src, radix_threshold(src, need, h, s_small), need, out + above, &s_count);
+    }
+}
+
+cudaError_t launch_topk_bracket(const Plan& p, const TopkArgs& a, cudaStream_t st) {
+    const cudaError_t e =
+        launch_pdl(topk_bracket_kernel, dim3(static_cast<unsigned>(p.rows_kv)), dim3(256), 0, st, a);
+    trace_mark("topk_bracket", st);
+    return e;
+}
+
+cudaError_t launch_topk_finalize(const Plan& p, const TopkArgs& a, cudaStream_t st) {
+    const cudaError_t e =
+        launch_pdl(topk_finalize_kernel<512>, dim3(static_cast<unsigned>(p.rows_kv)), dim3(512), 0, st, a);
+    trace_mark("topk_finalize", st);
+    return e;
+}
+
 cudaError_t launch_topk_rows(const Plan& p, const TopkArgs& a, cudaStream_t st) {
     const cudaError_t e =
         launch_pdl(topk_rows_kernel<512>, dim3(static_cast<unsigned>(p.rows_kv)), dim3(512), 0, st, a);

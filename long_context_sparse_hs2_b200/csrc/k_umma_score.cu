@@ -22,6 +22,7 @@
 // ring); warp 17 allocates TMEM and one of its lanes issues the MMAs.  Every wait is bounded; on expiry the CTA flags HS2_DEV_TIMEOUT, drains
 // and exits.
 #include "attn_sweep.cuh"
+#include "topk_common.cuh"
 #include "umma.cuh"
 
 namespace hs2 {
@@ -50,7 +51,9 @@ struct SSmem {
     static constexpr int kNumBars = 2 * kSStages + 5;    // kfull, kempty, sfull[2], tfree[2], done
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kPlOff = kMiscOff + 16;         // last pool key per query (-1: not ranked)
-    static constexpr int kBytes = kPlOff + kSMaxCols * 4 + 1024;
+    static constexpr int kBhiOff = kPlOff + kSMaxCols * 4;  // filter mode: each query's bracket bucket
+    static constexpr int kCntOff = kBhiOff + kSMaxCols * 4;  // filter mode: [warp][query] segment counts
+    static constexpr int kBytes = kCntOff + kSEpiWarps * (kSMaxCols / 4) * 4 + 1024;
 };
 
 __device__ __forceinline__ float max_nan(float a, float b) {
@@ -108,6 +111,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
     int* s_pl = reinterpret_cast<int*>(smem + L::kPlOff);
+    int* s_bhi = reinterpret_cast<int*>(smem + L::kBhiOff);
+    const int mode = a.score_mode;
+    const int tstep = mode == 1 ? kSampleTileStride : 1;  // sample mode: one tile in kSampleTileStride
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_trigger();
@@ -159,7 +165,15 @@ __global__ void __launch_bounds__(kSThreads, 1)
         fence_barrier_init();
     }
     pdl_wait();  // LSE_full comes from the previous kernel; TMEM only after it has completed
-    __syncthreads();  // s_pl complete
+    if (mode == 2) {  // the bracket of every query's selection row (written by the bracket kernel)
+        for (int qa = tid; qa < nq * TQ; qa += kSThreads) {
+            const int s = qa / TQ, tq = qa % TQ;
+            const int qb = split_keys ? pr : 2 * pr + s;
+            const int t = qb * TQ + tq;
+            s_bhi[qa] = (s_pl[qa] >= 0) ? a.meta[(static_cast<int64_t>(bh) * a.T + t) * kMetaInts + kMetaBin] : -1;
+        }
+    }
+    __syncthreads();  // s_pl (and s_bhi) complete
     const float sqrt_d = sqrtf(static_cast<float>(D));
     for (int i = tid; i < kSMaxCols * 8; i += kSThreads) {  // row block: -u as hi + mid + lo
         const int R = i >> 3, c = i & 7;
@@ -192,7 +206,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
 
     int jmax = -1;
     for (int qa = 0; qa < nq * TQ; ++qa) jmax = max(jmax, s_pl[qa]);
-    const int ntiles = jmax >= 0 ? (jmax + kSTile) / kSTile : 0;
+    // tiles (of the sample in sample mode: tile v stands for key tile v * tstep)
+    const int ntiles = jmax >= 0 ? ((jmax + kSTile) / kSTile + tstep - 1) / tstep : 0;
     const int t_begin = static_cast<int>((static_cast<int64_t>(split) * ntiles) / a.S);
     const int t_end = static_cast<int>((static_cast<int64_t>(split + 1) * ntiles) / a.S);
     const int nt = t_end - t_begin;
@@ -215,7 +230,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
                 for (int hb = 0; hb < D / 64; ++hb)
                     tma_load_3d(smem + L::kKOff + st * L::kTileBytes + hb * L::kBlock, &tmK, &kfull[st], hb * 64,
-                                (t_begin + q) * kSTile, bh, pol);
+                                (t_begin + q) * tstep * kSTile, bh, pol);
                 ++issued;
             }
             for (int st = 0; st < kSStages && st < issued; ++st) {
@@ -271,16 +286,24 @@ __global__ void __launch_bounds__(kSThreads, 1)
         for (int i = 0; i < nqw; ++i) plmin = min(plmin, s_pl[qa0 + i]);  // -1 if any is not ranked
         const uint32_t tbase = tm + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
         const float c2 = a.scale_log2;
+        // filter mode: this warp's segment (split, lane quarter) of every query's list, and its counts
+        int* s_cnt = reinterpret_cast<int*>(smem + L::kCntOff) + warp * (kSMaxCols / 4);
+        unsigned long long* seg = a.cand + (split * 4 + quarter) * a.seg_cap;
+        if (mode == 2) {
+            for (int i = lane; i < nqw; i += 32) s_cnt[i] = 0;
+            __syncwarp();
+        }
         for (int i = 0; i < nt; ++i) {
             const int buf = i & 1;
             const bool got = mbar_wait(&sfull[buf], (i >> 1) & 1, a.status);
             if (!got) *abort_flag = 1;
             if (!__all_sync(0xffffffffu, got && !*abort_flag)) break;
             tc_fence_after();
-            const int jt = (t_begin + i) * kSTile;
+            const int jt = (t_begin + i) * tstep * kSTile;  // first key of the tile
             const int j = jt + r;
             const bool fast = jt + kSTile - 1 <= plmin;  // every query of these columns takes every key
-            uint32_t* kp = a.keys + row0 * a.kstride + j;
+            // sample mode stores the tile compactly (tile i of the sample at i * 128)
+            uint32_t* kp = a.keys + row0 * a.kstride + (mode == 1 ? (t_begin + i) * kSTile + r : j);
             // read all of this warpgroup's columns, then hand the accumulator back to the MMA
             // before the max / key conversion / stores
             uint32_t x[2][32];
@@ -306,6 +329,26 @@ __global__ void __launch_bounds__(kSThreads, 1)
                     nonfinite |= (sv != sv) && (fast || j <= s_pl[qa0 + (32 * cq) / G + qq]);
                     key[qq] = score_key(sv);
                 }
+                if (mode == 2) {
+                    // each query's keys at or above its bracket bucket go to this warp's own segment
+                    // of the query's candidate list (a running count per warp and query in shared
+                    // memory: no atomics)
+#pragma unroll
+                    for (int qq = 0; qq < 32 / G; ++qq) {
+                        const int ql = (32 * cq) / G + qq;  // query of the warpgroup
+                        const int qa = qa0 + ql;
+                        const bool take = (fast || j <= s_pl[qa]) && score_bin(key[qq]) <= s_bhi[qa];
+                        const unsigned bal = __ballot_sync(0xffffffffu, take);
+                        if (bal == 0u) continue;
+                        const int c0 = s_cnt[ql];
+                        const int slot = c0 + __popc(bal & ((1u << lane) - 1u));
+                        if (take && slot < a.seg_cap) seg[(row0 + ql) * a.cand_cap + slot] = composite(key[qq], j);
+                        __syncwarp();
+                        if (lane == 0) s_cnt[ql] = c0 + __popc(bal);
+                        __syncwarp();
+                    }
+                    continue;
+                }
                 uint32_t* kq = kp + static_cast<int64_t>((32 * cq) / G) * a.kstride;
                 if (fast) {  // every query of these columns takes this key
 #pragma unroll
@@ -316,6 +359,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
                         if (j <= s_pl[qa0 + (32 * cq) / G + qq]) __stcs(kq + static_cast<int64_t>(qq) * a.kstride, key[qq]);
                 }
             }
+        }
+        if (mode == 2) {  // the segment counts of the ranked queries
+            __syncwarp();
+            for (int i = lane; i < nqw; i += 32)
+                if (s_pl[qa0 + i] >= 0) a.segcnt[(row0 + i) * (4 * a.S) + split * 4 + quarter] = s_cnt[i];
         }
     }
 
@@ -341,7 +389,7 @@ cudaError_t umma_score_variant(const Plan& p, const CUtensorMap& tmK, const Attn
     AttnArgs x = a;
     x.S = p.SS;
     e = launch_pdl(kern, grid, dim3(kSThreads), L::kBytes, st, tmK, x, split_keys);
-    trace_mark("umma_score", st);
+    trace_mark(a.score_mode == 1 ? "umma_score_sample" : (a.score_mode == 2 ? "umma_score_filter" : "umma_score"), st);
     return e;
 }
 

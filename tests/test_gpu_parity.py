@@ -80,6 +80,7 @@ CASES = [
     (1, 8, 1, 64, 3000, 40, 64, 32),      # several row blocks with a ragged last block
     (1, 4, 1, 128, 300, 1, 0, 16),        # k = 0: window only
     (1, 4, 1, 128, 300, 2, 10000, 16),    # k >= pool: collapses to full attention
+    (1, 4, 1, 128, 300, 1, 10000, 16),    # k >= pool at T = 1: the whole pool in index order
 ]
 
 
@@ -100,6 +101,14 @@ def test_positions_before_the_window_and_first_token():
     inp.k, inp.W = 3, 0
     res = run_step(inp)
     compare_step(inp, res)
+
+
+def test_decode_rows_at_scattered_positions():
+    # T = 1 (the one-launch decode step): per batch row the first token, an empty pool (pos < W),
+    # the pool's first key, and deep positions
+    pos = np.array([[0], [3], [63], [64], [999], [517]], np.int32)
+    inp = make_inputs(6, 8, 2, 128, 1000, 1, 16, 64, seed=15, needles=3, pos=pos)
+    compare_step(inp, run_step(inp))
 
 
 def test_empty_selection_gives_zero_output():
@@ -228,20 +237,25 @@ def test_repeated_calls_reuse_workspace():
 TAIL_CASES = [c for c in CASES if c[5] * (c[1] // c[2]) <= 16]
 
 
-@pytest.mark.parametrize("cluster", ["1", "0"], ids=["cluster_tail", "kernel_chain"])
+@pytest.mark.parametrize("path", ["fused", "cluster", "chain"])
 @pytest.mark.parametrize("case", TAIL_CASES, ids=[str(c) for c in TAIL_CASES])
-def test_decode_tail_paths_match_oracle(case, cluster, monkeypatch):
-    # decode shapes run the selection and the sparse layer in one cluster kernel; the kernel
-    # chain (score_hist -> topk_select -> sparse_attn) stays for shapes the cluster plan does not
-    # fit (a million-token pool) and is checked here too (HS2_CLUSTER_TAIL=0)
-    monkeypatch.setenv("HS2_CLUSTER_TAIL", cluster)
+def test_decode_tail_paths_match_oracle(case, path, monkeypatch):
+    # decode shapes (T = 1) run the whole step in one cooperative launch by default; the cluster
+    # tail (selection + sparse layer in one cluster kernel after the sweep) and the kernel chain
+    # (score_hist -> topk_select -> sparse_attn) remain for shapes the one-launch plan does not
+    # fit, and both are checked here too (HS2_FUSED_DECODE=0 with HS2_CLUSTER_TAIL=1 / 0)
+    if path != "fused":
+        monkeypatch.setenv("HS2_FUSED_DECODE", "0")
+        monkeypatch.setenv("HS2_CLUSTER_TAIL", "1" if path == "cluster" else "0")
     B, Hq, Hkv, d, N, T, k, W = case
     inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 7, needles=4)
     hs2.trace_enable(True)
     res = run_step(inp)
     kernels = hs2.trace_collect()
     hs2.trace_enable(False)
-    if cluster == "1":
+    if path == "fused":
+        assert ("decode_fused" in kernels) == (T == 1), kernels
+    elif path == "cluster":
         assert "select_sparse_cluster" in kernels and "topk_select" not in kernels, kernels
     else:
         assert "select_sparse_cluster" not in kernels and "topk_select" in kernels, kernels

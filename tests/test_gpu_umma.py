@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from long_context_sparse_hs2_b200 import hs2
-from long_context_sparse_hs2_b200.inputs import make_inputs
+from long_context_sparse_hs2_b200.inputs import f32_to_bf16_bits, make_inputs
 import oracle.hs2_oracle as O
 from tests import parity
 
@@ -136,30 +136,72 @@ def test_many_rows_all_scores_equal():
         np.testing.assert_array_equal(np.sort(res["idx"][b, h, t][:res["cnt"][b, h, t]]), r.selected)
 
 
-def test_many_rows_large_pools_sample_bracket():
-    # pools >= 32768 keys: the row top-k brackets the threshold from a 1/16 sample and selects
-    # in one pass; checked on sampled rows against the oracle and on every row's invariants
+@pytest.mark.parametrize("bracket", ["1", "0"], ids=["unstored_keys", "stored_keys"])
+def test_many_rows_large_pools_sample_bracket(bracket, monkeypatch):
+    # pools >= 32768 keys and >= 592 rows.  Default: the keys are never stored -- a 1/16 tile
+    # sample brackets each row's threshold, a filtering sweep keeps the candidates, and the
+    # exact top-k is taken among them.  HS2_PREFILL_BRACKET=0 stores every key and brackets
+    # inside the one-CTA-per-row top-k.  Sampled rows against the oracle, every row's invariants.
     from tests.test_gpu_parity import compare_step, run_step
     from tests.test_gpu_workloads import check_all_rows
 
+    monkeypatch.setenv("HS2_PREFILL_BRACKET", bracket)
     inp = make_inputs(1, 8, 1, 128, 40000, 600, 2048, 128, seed=23, needles=32)
-    res = run_step(inp)
+    g = parity.gpu_inputs(inp)
+    ws = hs2.alloc_workspace(hs2.dims_of(g["Q_full"], g["K"], inp.k, inp.W), "cuda")
+    hs2.trace_enable(True)
+    res = run_step(inp, ws)
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    if bracket == "1":
+        assert "topk_bracket" in kernels and "topk_finalize" in kernels and "topk_rows" not in kernels, kernels
+        # N(0, 1) scores: the sample brackets every row, no row is rescored
+        assert hs2.read_device_status(ws) == 0
+    else:
+        assert "topk_rows" in kernels and "topk_bracket" not in kernels, kernels
     check_all_rows(inp, res["idx"], res["cnt"])
     compare_step(inp, res, rows=[(0, 0, t) for t in (0, 1, 77, 300, 301, 598, 599)])
 
 
 def test_many_rows_large_pools_all_ties_fall_back():
-    # every score equal: the sample cannot bracket the threshold within shared memory, so the
-    # exact two-pass method runs (and re-scans the keys for the tied bucket)
+    # every score equal: all pool keys share one bucket, the candidate list overflows, and each
+    # row is rescored on the CUDA cores with the exact two-pass method (recomputing the tied
+    # bucket's keys on every radix pass); flagged HS2_DEV_CAND_OVERFLOW
     from tests.test_gpu_parity import compare_step, run_step
 
     inp = make_inputs(1, 8, 1, 128, 40000, 600, 500, 64, seed=24)
     inp.Qf = np.zeros_like(inp.Qf)
-    res = run_step(inp)
+    g = parity.gpu_inputs(inp)
+    ws = hs2.alloc_workspace(hs2.dims_of(g["Q_full"], g["K"], inp.k, inp.W), "cuda")
+    res = run_step(inp, ws)
+    assert hs2.read_device_status(ws) == hs2.DEV_CAND_OVERFLOW
     rows = [(0, 0, t) for t in (0, 299, 599)]
     ref = compare_step(inp, res, rows=rows)
     for (b, h, t), r in ref.items():
         np.testing.assert_array_equal(np.sort(res["idx"][b, h, t][:res["cnt"][b, h, t]]), r.selected)
+
+
+@pytest.mark.parametrize("factor", [3.0, 0.25], ids=["sample_too_strict", "sample_too_loose"])
+def test_many_rows_large_pools_misleading_sample(factor):
+    # K scaled by `factor` in exactly the sampled 128-key tiles (every 16th): the sample's
+    # estimate of each row's k-th best score is far off, so the candidate list holds fewer
+    # than k keys (factor 3) or overflows (factor 1/4), and every ranked row is rescored
+    # exactly.  Sampled rows against the oracle, every row's invariants.
+    from tests.test_gpu_parity import compare_step, run_step
+    from tests.test_gpu_workloads import check_all_rows
+    from long_context_sparse_hs2_b200.inputs import bf16_bits_to_f32
+
+    inp = make_inputs(1, 8, 1, 128, 40000, 600, 2048, 128, seed=26)
+    kk = bf16_bits_to_f32(inp.K)
+    tiles = (np.arange(kk.shape[2]) // 128) % 16 == 0
+    kk[:, :, tiles] *= np.float32(factor)
+    inp.K = f32_to_bf16_bits(kk)
+    g = parity.gpu_inputs(inp)
+    ws = hs2.alloc_workspace(hs2.dims_of(g["Q_full"], g["K"], inp.k, inp.W), "cuda")
+    res = run_step(inp, ws)
+    assert hs2.read_device_status(ws) == hs2.DEV_CAND_OVERFLOW
+    check_all_rows(inp, res["idx"], res["cnt"])
+    compare_step(inp, res, rows=[(0, 0, t) for t in (0, 150, 599)])
 
 
 def test_multi_cta_topk_with_several_chunks_per_cta():
