@@ -136,12 +136,14 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     // kernel's combine CTA G * S1 weights in its histogram scratch
     if (static_cast<int64_t>(G) * P.S4 > 8192 || static_cast<int64_t>(G) * P.S1 > 4096) return false;
     P.cand_cap = std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
-    // one-launch decode step: one selection row per row block, kept logits, every candidate list
-    // able to hold a whole pool, a split's pool keys within the kernel's shared-memory key buffer
+    // one-launch decode step (HS2_FUSED_DECODE=1; it measured slower than the kernel chain at every
+    // decode shape: its row barriers and per-CTA latency chains cost more than the launches they
+    // save): one selection row per row block, kept logits, every candidate list able to hold a
+    // whole pool, a split's pool keys within the kernel's shared-memory key buffer
     const char* want_fused = std::getenv("HS2_FUSED_DECODE");
     const int64_t tiles64 = (static_cast<int64_t>(x.N) + kKeyTile - 1) / kKeyTile;
     P.fused = x.T == 1 && P.RT == 1 && P.mat_logits && !P.umma && P.cand_cap >= x.N &&
-              ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap && !(want_fused && want_fused[0] == '0');
+              ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap && want_fused && want_fused[0] == '1';
     const int64_t sparse_slots = P.fused ? std::max<int64_t>(P.S4, P.S1) : P.S4;
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
     // bracketed selection (tcgen05 score sweep, many rows, large pools): a 1/16 tile sample per

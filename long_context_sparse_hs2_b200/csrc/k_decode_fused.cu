@@ -7,7 +7,7 @@
 //      partial (m, l, O) of the row's G heads and the kept base-2 logits of its keys;
 //   -- row barrier: every split of the row has published its partial --
 //   2. merges the G heads' LSE from the S partials (every CTA, the same fixed order, so all get
-//      bit-identical values) and writes its share of the O_full / LSE_full combine;
+//      bit-identical values) and writes its 1/S share of the O_full / LSE_full columns;
 //   3. scores its own pool keys from the kept logits (max over heads of logit - LSE, as
 //      order-preserving keys in shared memory) and adds its histogram to the row's;
 //   -- row barrier: the row's histogram is complete --
@@ -15,13 +15,16 @@
 //      writes its keys of better buckets to the index list and its keys of b1 to the row's
 //      candidate list (one 64-bit atomic per CTA reserves both ranges);
 //   -- row barrier: the candidate list is complete --
-//   5. radix-selects the exact threshold composite among the candidates (every CTA, identical
-//      result) and writes its own candidates at or above it;
+//   5. ranks each of its own candidates against the whole list (a candidate is selected iff
+//      fewer than keff - above others beat it, and that rank is its slot), or, for a long list,
+//      radix-selects the exact threshold composite (every CTA, identical) and writes its own
+//      candidates at or above it;
 //   -- row barrier: the row's index list (window, selection, padding) is complete --
 //   6. runs the sparse layer over an equal share of the index list: the rows gathered with
 //      16-byte cp.async into the swizzled tile layout (two 64-key stages), the same warp
 //      attention core as the sweep, one split partial per CTA;
-//   7. the row's last CTA (a completion counter; nothing waits) merges the S sparse partials.
+//   -- row barrier: every sparse partial is written --
+//   7. merges its share of the outputs' columns from the S sparse partials.
 // The selection rule is that of the kernel chain (ties to the lower index, NaN ranked last); the
 // split-K partials and the log-sum-exp merges are those of "Simplified Sparse Attention via Gist
 // Tokens", section 3.6.  A row barrier is an arrival counter per row and a bounded spin
@@ -42,7 +45,8 @@ constexpr int kFNC = 4;                    // consumer warps (four 16-key slices
 constexpr int kFWarps = kFNC + 1;          // + the TMA producer of the sweep
 constexpr int kFThreads = kFWarps * 32;
 constexpr int kFKeyCap = kFusedKeyCap;     // pool keys of one split kept in shared memory
-constexpr int kFCandCap = 2048;            // candidates radix-selected from shared memory
+constexpr int kFCandCap = 2048;            // a row's candidates ranked from shared memory
+constexpr int kFOwnCap = 1024;             // a CTA's own candidates kept in shared memory
 
 template <int D, int STAGES, bool FP8>
 struct FSmem {
@@ -181,6 +185,82 @@ __device__ __forceinline__ void gather_stage(const void* K, const void* V, const
     }
 }
 
+// Merges the S split partials (m, l, acc) of the G query-head rows row0 .. row0 + G - 1 (every CTA
+// computes the same per-split weights, in one fixed order) and writes this CTA's contiguous share
+// of the outputs' float4 columns (split of S): bf16 O and, with a row's first column, its
+// natural-log LSE; s_lse2 receives each head's base-2 LSE.  Every (column, split) product is
+// loaded by its own thread, and the products are summed in a fixed order, so the result does not
+// depend on timing.  scratch: G * S float2 + G * S floats + ceil(G*D/4 / S) * S float4 bytes of
+// shared memory.  Call from all threads.
+template <int D, int G>
+__device__ __forceinline__ void merge_share(const float2* __restrict__ part_ml, const float* __restrict__ part_acc,
+                                            int S, int64_t rows, int64_t row0, int split, uint8_t* scratch,
+                                            float2* s_ml, float* s_lse2, uint16_t* O, float* LSE) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+    float2* s_pml = reinterpret_cast<float2*>(scratch);               // [G][S]
+    float* s_w = reinterpret_cast<float*>(s_pml + G * S);              // [G][S]
+    float4* s_prod = reinterpret_cast<float4*>(s_w + ((G * S + 3) & ~3));  // [columns of this CTA][S]
+    for (int e = tid; e < G * S; e += blockDim.x) {
+        const int g = e / S, sp = e % S;
+        s_pml[e] = __ldcg(&part_ml[static_cast<int64_t>(sp) * rows + row0 + g]);
+    }
+    __syncthreads();
+    for (int g = warp; g < G; g += nw) {
+        const float2* pm = s_pml + g * S;
+        float m = -INFINITY;
+        for (int sp = lane; sp < S; sp += 32) m = fmaxf(m, pm[sp].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
+        if (m != -INFINITY)
+            for (int sp = lane; sp < S; sp += 32)
+                if (pm[sp].x != -INFINITY) l += fast_exp2(pm[sp].x - m) * pm[sp].y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        for (int sp = lane; sp < S; sp += 32)
+            s_w[g * S + sp] = (pm[sp].x == -INFINITY || m == -INFINITY) ? 0.f : fast_exp2(pm[sp].x - m) * inv;
+        if (lane == 0) {
+            s_ml[g] = make_float2(m, l);
+            s_lse2[g] = lse2_of(make_float2(m, l));
+        }
+    }
+    __syncthreads();
+    constexpr int C4 = D / 4;
+    const int ncol = G * C4;
+    const int c_lo = static_cast<int>((static_cast<int64_t>(split) * ncol) / S);
+    const int c_hi = static_cast<int>((static_cast<int64_t>(split + 1) * ncol) / S);
+    const int nc = c_hi - c_lo;
+    for (int e = tid; e < nc * S; e += blockDim.x) {
+        const int cl = e / S, sp = e % S;
+        const int col = c_lo + cl, g = col / C4, c = col % C4;
+        const float wt = s_w[g * S + sp];
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (wt != 0.f) {
+            x = __ldcg(reinterpret_cast<const float4*>(part_acc + ((static_cast<int64_t>(sp) * rows + row0 + g) * D + c * 4)));
+            x = make_float4(wt * x.x, wt * x.y, wt * x.z, wt * x.w);
+        }
+        s_prod[e] = x;
+    }
+    __syncthreads();
+    for (int cl = tid; cl < nc; cl += blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < S; ++sp) {
+            const float4 x = s_prod[cl * S + sp];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        const int col = c_lo + cl, g = col / C4, c = col % C4;
+        const int64_t row = row0 + g;
+        *reinterpret_cast<uint2*>(O + row * D + c * 4) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        if (c == 0) LSE[row] = s_lse2[g] * kLn2;
+    }
+    __syncthreads();
+}
+
 }  // namespace
 
 template <int D, int G, int STAGES, bool FP8>
@@ -197,7 +277,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
     __shared__ unsigned s_small[2];
     __shared__ unsigned s_warp[32];
     __shared__ unsigned long long s_base2;
-    __shared__ int s_int[8];  // 0 barrier flag, 1 b1, 2 above, 3 last CTA, 4 reserved base
+    __shared__ int s_int[8];  // 0 barrier flag, 1 b1, 2 above, 4 reserved base, 5 own candidates
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, row = blockIdx.y, S = gridDim.x;  // row = b * Hkv + h
@@ -220,19 +300,9 @@ __global__ void __launch_bounds__(kFThreads, 2)
     pdl_trigger();  // every CTA of the grid is resident and past its sweep
 
     // ---- 2. the G heads' LSE (every CTA) and this CTA's share of the O_full combine
-    float* s_w = reinterpret_cast<float*>(smem + L::kCandOff);  // G * S <= 4096 merge weights
-    if (ok) {
-        for (int g = warp; g < G; g += kFWarps) {
-            const float2 ML = warp_row_weights(a.part_ml, S, rows_q, rq0 + g, s_w + g * S);
-            if (lane == 0) {
-                s_ml[g] = ML;
-                s_lse2[g] = lse2_of(ML);
-            }
-        }
-        __syncthreads();
-        combine_columns<D, 8>(a.part_acc, S, rows_q, rq0, 1, G, s_w, s_ml, f.O_full, f.LSE_full,
-                              split * kFThreads + tid, S * kFThreads);
-    }
+    if (ok)
+        merge_share<D, G>(a.part_ml, a.part_acc, S, rows_q, rq0, split, smem + L::kKeysOff, s_ml, s_lse2, f.O_full,
+                          f.LSE_full);
 
     const int pos = clamp_pos(a.pos[b], a.N, nullptr);  // a bad position was flagged by the sweep
     const int P = max(0, pos - a.W + 1);                 // pool: keys 0 .. pos - W
@@ -244,6 +314,8 @@ __global__ void __launch_bounds__(kFThreads, 2)
     int32_t* idx = f.idx + static_cast<int64_t>(row) * kw;
     uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + L::kKeysOff);
     unsigned* s_hist = reinterpret_cast<unsigned*>(smem + L::kHistOff);
+    // this CTA's candidates (the threshold bucket's keys), over the histogram once b1 is known
+    unsigned long long* s_own = reinterpret_cast<unsigned long long*>(smem + L::kHistOff);
 
     if (ranked) {
         // ---- 3. scores of this CTA's pool keys, local histogram into the row's
@@ -256,7 +328,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
             for (int g = 0; g < G; ++g) lse[g] = s_lse2[g];
             const float* lg = a.logits + static_cast<int64_t>(row) * a.N * G;
             bool nonfinite = false;
-            constexpr int U = 4;  // keys in flight per thread
+            constexpr int U = G >= 16 ? 4 : 8;  // keys in flight per thread
             for (int base = tid; base < nown; base += U * kFThreads) {
                 float v[U][G];
 #pragma unroll
@@ -307,8 +379,27 @@ __global__ void __launch_bounds__(kFThreads, 2)
                 s_int[2] = 0;
             }
             __syncthreads();
-            if (warp == 0) warp_bucket_at(s_hist, static_cast<unsigned>(keff), &s_int[1], &s_int[2]);
-            __syncthreads();
+            {  // the bucket holding the keff-th best key: 16 buckets per thread over 128 threads
+                constexpr int PER = kHistBins / 128;
+                unsigned v = 0;
+                if (tid < 128)
+                    for (int i = 0; i < PER; ++i) v += s_hist[tid * PER + i];
+                const unsigned excl = block_exclusive_scan(v, s_warp);
+                const unsigned need = static_cast<unsigned>(keff);
+                if (tid < 128 && excl < need && need <= excl + v) {
+                    unsigned cum = excl;
+                    for (int i = 0; i < PER; ++i) {
+                        const unsigned x = s_hist[tid * PER + i];
+                        if (cum + x >= need) {
+                            s_int[1] = tid * PER + i;
+                            s_int[2] = static_cast<int>(cum);
+                            break;
+                        }
+                        cum += x;
+                    }
+                }
+                __syncthreads();
+            }
             const int b1 = s_int[1], above = s_int[2];
             unsigned nd = 0, nc = 0;
             for (int i = tid; i < nown; i += kFThreads) {
@@ -316,11 +407,12 @@ __global__ void __launch_bounds__(kFThreads, 2)
                 nd += bin < b1;
                 nc += bin == b1;
             }
-            unsigned td, tc;
-            const unsigned ed = block_scan_total(nd, s_warp, &td);
-            const unsigned ec = block_scan_total(nc, s_warp, &tc);
-            const int2 base = block_reserve2(static_cast<int>(td), static_cast<int>(tc), meta + kMetaDef, &s_base2);
-            int od = base.x + static_cast<int>(ed), oc = base.y + static_cast<int>(ec);
+            unsigned tot;
+            const unsigned ex = block_scan_total(nd | (nc << 16), s_warp, &tot);  // both < 2^16 per CTA
+            const int td = static_cast<int>(tot & 0xFFFFu), tc = static_cast<int>(tot >> 16);
+            const int2 base = block_reserve2(td, tc, meta + kMetaDef, &s_base2);
+            int od = base.x + static_cast<int>(ex & 0xFFFFu), oc = base.y + static_cast<int>(ex >> 16);
+            int lo_own = static_cast<int>(ex >> 16);
             unsigned long long* gc = f.cand + static_cast<int64_t>(row) * f.cand_cap;
             for (int i = tid; i < nown; i += kFThreads) {
                 const uint32_t key = s_keys[i];
@@ -329,42 +421,62 @@ __global__ void __launch_bounds__(kFThreads, 2)
                     if (od < above) idx[wcnt + od] = j_lo + i;
                     ++od;
                 } else if (bin == b1) {
-                    if (oc < f.cand_cap) gc[oc] = composite(key, j_lo + i);
+                    const unsigned long long c = composite(key, j_lo + i);
+                    if (oc < f.cand_cap) gc[oc] = c;
+                    if (lo_own < kFOwnCap) s_own[lo_own] = c;
                     ++oc;
+                    ++lo_own;
                 }
             }
+            if (tid == 0) s_int[5] = tc;
         }
         ok = row_barrier(bar_ctr, (++arrivals) * S, a.status, ok, &s_int[0]);
 
-        // ---- 5. exact threshold among the candidates (every CTA); this CTA's winners out
+        // ---- 5. the winners among the candidates: a candidate is selected iff fewer than
+        // need = keff - above candidates beat it (composites are distinct), and its rank is its
+        // slot.  Every CTA ranks its own candidates against the whole list; a longer list (heavy
+        // ties) takes the exact radix threshold instead, in every CTA of the row alike.
         if (ok) {
-            const int b1 = s_int[1], above = s_int[2];
+            const int above = s_int[2], b1 = s_int[1], own = min(s_int[5], kFOwnCap);
             const unsigned need = static_cast<unsigned>(keff - above);
-            const int64_t nc = __ldcg(meta + kMetaCand);
-            const int n = static_cast<int>(nc < f.cand_cap ? nc : f.cand_cap);
+            const int64_t ncand = __ldcg(meta + kMetaCand);
+            const int n = static_cast<int>(ncand < f.cand_cap ? ncand : f.cand_cap);
             const unsigned long long* gc = f.cand + static_cast<int64_t>(row) * f.cand_cap;
-            unsigned long long thr;
-            if (n <= kFCandCap) {
-                unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(smem + L::kCandOff);
+            unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(smem + L::kCandOff);
+            if (n <= kFOwnCap) {  // row-uniform: then every CTA holds all its own candidates
                 for (int i = tid; i < n; i += kFThreads) s_cand[i] = __ldcg(gc + i);
                 __syncthreads();
-                thr = radix_threshold(SmemSource{s_cand, n}, need, s_hh, s_small);
+                for (int o = warp; o < own; o += kFWarps) {
+                    const unsigned long long c = s_own[o];
+                    int r = 0;
+                    for (int i = lane; i < n; i += 32) r += s_cand[i] > c;
+#pragma unroll
+                    for (int x = 16; x > 0; x >>= 1) r += __shfl_xor_sync(0xffffffffu, r, x);
+                    if (lane == 0 && r < static_cast<int>(need)) idx[wcnt + above + r] = composite_index(c);
+                }
             } else {
-                thr = radix_threshold(GlobalSource{gc, n}, need, s_hh, s_small);
-            }
-            unsigned ns = 0;
-            for (int i = tid; i < nown; i += kFThreads) {
-                const uint32_t key = s_keys[i];
-                ns += score_bin(key) == b1 && composite(key, j_lo + i) >= thr;
-            }
-            unsigned ts;
-            const unsigned es = block_scan_total(ns, s_warp, &ts);
-            int o = block_reserve(static_cast<int>(ts), meta + kMetaAbove, &s_int[4]) + static_cast<int>(es);
-            for (int i = tid; i < nown; i += kFThreads) {
-                const uint32_t key = s_keys[i];
-                if (score_bin(key) == b1 && composite(key, j_lo + i) >= thr) {
-                    if (o < static_cast<int>(need)) idx[wcnt + above + o] = j_lo + i;
-                    ++o;
+                unsigned long long thr;
+                if (n <= kFCandCap) {
+                    for (int i = tid; i < n; i += kFThreads) s_cand[i] = __ldcg(gc + i);
+                    __syncthreads();
+                    thr = radix_threshold(SmemSource{s_cand, n}, need, s_hh, s_small);
+                } else {
+                    thr = radix_threshold(GlobalSource{gc, n}, need, s_hh, s_small);
+                }
+                unsigned ns = 0;
+                for (int i = tid; i < nown; i += kFThreads) {
+                    const uint32_t key = s_keys[i];
+                    ns += score_bin(key) == b1 && composite(key, j_lo + i) >= thr;
+                }
+                unsigned ts;
+                const unsigned es = block_scan_total(ns, s_warp, &ts);
+                int o = block_reserve(static_cast<int>(ts), meta + kMetaAbove, &s_int[4]) + static_cast<int>(es);
+                for (int i = tid; i < nown; i += kFThreads) {
+                    const uint32_t key = s_keys[i];
+                    if (score_bin(key) == b1 && composite(key, j_lo + i) >= thr) {
+                        if (o < static_cast<int>(need)) idx[wcnt + above + o] = j_lo + i;
+                        ++o;
+                    }
                 }
             }
         }
@@ -457,17 +569,11 @@ __global__ void __launch_bounds__(kFThreads, 2)
         __syncthreads();
         merge_states<D, kFNC>(red, tid, kFThreads, out, row_q);
     }
+    ok = row_barrier(bar_ctr, (++arrivals) * S, a.status, ok, &s_int[0]);
 
-    // ---- 7. the row's last CTA merges the sparse partials
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_int[3] = atomicAdd(meta + kMetaSparseDone, 1) == S - 1;
-    __syncthreads();
-    if (!s_int[3]) return;
-    __threadfence();
-    float* w2 = reinterpret_cast<float*>(smem);  // G * S weights, then the (m, l)
-    float2* ml2 = reinterpret_cast<float2*>(smem + L::kCandOff);
-    block_combine_rows<D>(f.ps_ml, f.ps_acc, S, rows_q, rq0, 1, G, w2, ml2, f.O_sparse, f.LSE_sparse);
+    // ---- 7. every CTA merges its share of the sparse partials
+    if (ok)
+        merge_share<D, G>(f.ps_ml, f.ps_acc, S, rows_q, rq0, split, smem, s_ml, s_lse2, f.O_sparse, f.LSE_sparse);
 }
 
 // ====================================================================== launcher

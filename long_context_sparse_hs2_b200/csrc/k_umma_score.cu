@@ -51,8 +51,8 @@ struct SSmem {
     static constexpr int kNumBars = 2 * kSStages + 5;    // kfull, kempty, sfull[2], tfree[2], done
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kPlOff = kMiscOff + 16;         // last pool key per query (-1: not ranked)
-    static constexpr int kBhiOff = kPlOff + kSMaxCols * 4;  // filter mode: each query's bracket bucket
-    static constexpr int kCntOff = kBhiOff + kSMaxCols * 4;  // filter mode: [warp][query] segment counts
+    static constexpr int kThrOff = kPlOff + kSMaxCols * 4;  // filter mode: each query's score bound
+    static constexpr int kCntOff = kThrOff + kSMaxCols * 4;  // filter mode: [warp][query] segment counts
     static constexpr int kBytes = kCntOff + kSEpiWarps * (kSMaxCols / 4) * 4 + 1024;
 };
 
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
     int* s_pl = reinterpret_cast<int*>(smem + L::kPlOff);
-    int* s_bhi = reinterpret_cast<int*>(smem + L::kBhiOff);
+    float* s_thr = reinterpret_cast<float*>(smem + L::kThrOff);
     const int mode = a.score_mode;
     const int tstep = mode == 1 ? kSampleTileStride : 1;  // sample mode: one tile in kSampleTileStride
 
@@ -165,12 +165,24 @@ __global__ void __launch_bounds__(kSThreads, 1)
         fence_barrier_init();
     }
     pdl_wait();  // LSE_full comes from the previous kernel; TMEM only after it has completed
-    if (mode == 2) {  // the bracket of every query's selection row (written by the bracket kernel)
+    if (mode == 2) {
+        // The bracket of every query's selection row (the bracket kernel's bucket b_hi) as a bound
+        // on the score itself: score_bin(key(s)) <= b_hi exactly when s > -F, F the float whose
+        // bits are (b_hi + 1) << 15 above the first bucket's (see score_bin).  b_hi = the last
+        // bucket takes every key except NaN and -inf, which rank below all others.
         for (int qa = tid; qa < nq * TQ; qa += kSThreads) {
             const int s = qa / TQ, tq = qa % TQ;
             const int qb = split_keys ? pr : 2 * pr + s;
             const int t = qb * TQ + tq;
-            s_bhi[qa] = (s_pl[qa] >= 0) ? a.meta[(static_cast<int64_t>(bh) * a.T + t) * kMetaInts + kMetaBin] : -1;
+            float thr = INFINITY;
+            if (s_pl[qa] >= 0) {
+                const int bhi = a.meta[(static_cast<int64_t>(bh) * a.T + t) * kMetaInts + kMetaBin];
+                if (bhi >= kHistBins - 1)
+                    thr = -INFINITY;
+                else if (bhi >= 0)
+                    thr = -__uint_as_float(static_cast<uint32_t>(bhi + (125 << 8) + 1) << 15);
+            }
+            s_thr[qa] = thr;
         }
     }
     __syncthreads();  // s_pl (and s_bhi) complete
@@ -286,10 +298,17 @@ __global__ void __launch_bounds__(kSThreads, 1)
         for (int i = 0; i < nqw; ++i) plmin = min(plmin, s_pl[qa0 + i]);  // -1 if any is not ranked
         const uint32_t tbase = tm + (static_cast<uint32_t>(quarter * 32) << 16) + col0;
         const float c2 = a.scale_log2;
-        // filter mode: this warp's segment (split, lane quarter) of every query's list, and its counts
+        // filter mode: this warp's segment (split, lane quarter) of every query's list, and its
+        // running counts (registers for G >= 4, shared memory otherwise)
         int* s_cnt = reinterpret_cast<int*>(smem + L::kCntOff) + warp * (kSMaxCols / 4);
         unsigned long long* seg = a.cand + (split * 4 + quarter) * a.seg_cap;
-        if (mode == 2) {
+        constexpr bool kRegCnt = G >= 4;
+        int qcnt[2][32 / G];
+#pragma unroll
+        for (int cq = 0; cq < 2; ++cq)
+#pragma unroll
+            for (int qq = 0; qq < 32 / G; ++qq) qcnt[cq][qq] = 0;
+        if (mode == 2 && !kRegCnt) {
             for (int i = lane; i < nqw; i += 32) s_cnt[i] = 0;
             __syncwarp();
         }
@@ -321,34 +340,39 @@ __global__ void __launch_bounds__(kSThreads, 1)
                 float m[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) m[e] = __uint_as_float(x[cq][e]);
-                uint32_t key[32 / G];
+                float sv[32 / G];
 #pragma unroll
                 for (int qq = 0; qq < 32 / G; ++qq) {
-                    const float sv = head_max<G>(m + qq * G) * c2;
+                    sv[qq] = head_max<G>(m + qq * G) * c2;
                     // only keys that are stored count (past a query's pool the slot may hold anything)
-                    nonfinite |= (sv != sv) && (fast || j <= s_pl[qa0 + (32 * cq) / G + qq]);
-                    key[qq] = score_key(sv);
+                    nonfinite |= (sv[qq] != sv[qq]) && (fast || j <= s_pl[qa0 + (32 * cq) / G + qq]);
                 }
                 if (mode == 2) {
-                    // each query's keys at or above its bracket bucket go to this warp's own segment
-                    // of the query's candidate list (a running count per warp and query in shared
-                    // memory: no atomics)
+                    // each query's keys above its score bound go to this warp's own segment of the
+                    // query's candidate list (a running count per warp and query: no atomics)
 #pragma unroll
                     for (int qq = 0; qq < 32 / G; ++qq) {
                         const int ql = (32 * cq) / G + qq;  // query of the warpgroup
-                        const int qa = qa0 + ql;
-                        const bool take = (fast || j <= s_pl[qa]) && score_bin(key[qq]) <= s_bhi[qa];
+                        const bool take = sv[qq] > s_thr[qa0 + ql] && (fast || j <= s_pl[qa0 + ql]);
                         const unsigned bal = __ballot_sync(0xffffffffu, take);
                         if (bal == 0u) continue;
-                        const int c0 = s_cnt[ql];
+                        const int c0 = kRegCnt ? qcnt[cq][qq] : s_cnt[ql];
                         const int slot = c0 + __popc(bal & ((1u << lane) - 1u));
-                        if (take && slot < a.seg_cap) seg[(row0 + ql) * a.cand_cap + slot] = composite(key[qq], j);
-                        __syncwarp();
-                        if (lane == 0) s_cnt[ql] = c0 + __popc(bal);
-                        __syncwarp();
+                        if (take && slot < a.seg_cap)
+                            seg[(row0 + ql) * a.cand_cap + slot] = composite(score_key(sv[qq]), j);
+                        if (kRegCnt) {
+                            qcnt[cq][qq] = c0 + __popc(bal);
+                        } else {
+                            __syncwarp();
+                            if (lane == 0) s_cnt[ql] = c0 + __popc(bal);
+                            __syncwarp();
+                        }
                     }
                     continue;
                 }
+                uint32_t key[32 / G];
+#pragma unroll
+                for (int qq = 0; qq < 32 / G; ++qq) key[qq] = score_key(sv[qq]);
                 uint32_t* kq = kp + static_cast<int64_t>((32 * cq) / G) * a.kstride;
                 if (fast) {  // every query of these columns takes this key
 #pragma unroll
@@ -361,9 +385,22 @@ __global__ void __launch_bounds__(kSThreads, 1)
             }
         }
         if (mode == 2) {  // the segment counts of the ranked queries
-            __syncwarp();
-            for (int i = lane; i < nqw; i += 32)
-                if (s_pl[qa0 + i] >= 0) a.segcnt[(row0 + i) * (4 * a.S) + split * 4 + quarter] = s_cnt[i];
+            if (kRegCnt) {
+                if (lane == 0) {
+#pragma unroll
+                    for (int cq = 0; cq < 2; ++cq)
+#pragma unroll
+                        for (int qq = 0; qq < 32 / G; ++qq) {
+                            const int ql = (32 * cq) / G + qq;
+                            if (ql < nqw && s_pl[qa0 + ql] >= 0)
+                                a.segcnt[(row0 + ql) * (4 * a.S) + split * 4 + quarter] = qcnt[cq][qq];
+                        }
+                }
+            } else {
+                __syncwarp();
+                for (int i = lane; i < nqw; i += 32)
+                    if (s_pl[qa0 + i] >= 0) a.segcnt[(row0 + i) * (4 * a.S) + split * 4 + quarter] = s_cnt[i];
+            }
         }
     }
 

@@ -224,6 +224,14 @@ def test_decode_loop_replayed_from_one_cuda_graph(dtype, page_size):
     _decode_run(dtype, page_size, seed=31 + page_size, graph=True)
 
 
+@pytest.mark.parametrize("dtype,page_size,graph", [("bf16", 0, False), ("fp8_e4m3", 16, False), ("bf16", 16, True)])
+def test_decode_loop_in_one_launch_per_step(dtype, page_size, graph, monkeypatch):
+    # the decode loop with each step in one cooperative launch (HS2_FUSED_DECODE=1): FP8 and paged
+    # caches, eager and replayed from one CUDA graph
+    monkeypatch.setenv("HS2_FUSED_DECODE", "1")
+    _decode_run(dtype, page_size, seed=41 + page_size, graph=graph)
+
+
 def test_decode_step_on_a_full_cache_keeps_its_position():
     # pos[b] + 1 == N: nothing is appended, pos stays, the bit is set and the step runs at N - 1
     inp = make_inputs(1, 8, 1, 128, 256, 1, 16, 8, seed=4, pos=np.array([[255]], np.int32))

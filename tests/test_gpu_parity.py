@@ -240,12 +240,12 @@ TAIL_CASES = [c for c in CASES if c[5] * (c[1] // c[2]) <= 16]
 @pytest.mark.parametrize("path", ["fused", "cluster", "chain"])
 @pytest.mark.parametrize("case", TAIL_CASES, ids=[str(c) for c in TAIL_CASES])
 def test_decode_tail_paths_match_oracle(case, path, monkeypatch):
-    # decode shapes (T = 1) run the whole step in one cooperative launch by default; the cluster
-    # tail (selection + sparse layer in one cluster kernel after the sweep) and the kernel chain
-    # (score_hist -> topk_select -> sparse_attn) remain for shapes the one-launch plan does not
-    # fit, and both are checked here too (HS2_FUSED_DECODE=0 with HS2_CLUSTER_TAIL=1 / 0)
-    if path != "fused":
-        monkeypatch.setenv("HS2_FUSED_DECODE", "0")
+    # the decode tail after the sweep: the cluster tail (selection + sparse layer in one cluster
+    # kernel), the kernel chain (score_hist -> topk_select -> sparse_attn), and, for T = 1, the
+    # whole step in one cooperative launch (HS2_FUSED_DECODE=1)
+    if path == "fused":
+        monkeypatch.setenv("HS2_FUSED_DECODE", "1")
+    else:
         monkeypatch.setenv("HS2_CLUSTER_TAIL", "1" if path == "cluster" else "0")
     B, Hq, Hkv, d, N, T, k, W = case
     inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 7, needles=4)

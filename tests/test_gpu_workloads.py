@@ -109,6 +109,22 @@ def test_workload_full_size(name):
     compare_step(inp, res, rows=SAMPLES[name])
 
 
+@pytest.mark.parametrize("name", ["long", "1m_t1"])
+def test_workload_full_size_one_launch_decode(name, monkeypatch):
+    # the whole decode step in one cooperative launch (opt-in), at full size: every row's
+    # selection invariants and the sampled rows against the oracle
+    monkeypatch.setenv("HS2_FUSED_DECODE", "1")
+    w = WORKLOADS[name]
+    inp = generate(w)
+    hs2.trace_enable(True)
+    res = _run(inp, w)
+    kernels = hs2.trace_collect()
+    hs2.trace_enable(False)
+    assert "decode_fused" in kernels, kernels
+    check_all_rows(inp, res["idx"], res["cnt"])
+    compare_step(inp, res, rows=SAMPLES[name])
+
+
 @pytest.mark.parametrize("name", list(VARIANTS))
 def test_workload_cache_variant_full_size(name):
     base, dtype, page_size = VARIANTS[name]
