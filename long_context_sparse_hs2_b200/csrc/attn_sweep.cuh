@@ -12,7 +12,7 @@
 // without reading K a second time.
 #pragma once
 
-#include "attn_core.cuh"
+#include "attn_core_t.cuh"
 
 namespace hs2 {
 
@@ -117,13 +117,15 @@ __device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, ui
 // split's K/V tiles through the TMA ring, keeps the online softmax, optionally stores the
 // base-2 logits, and writes the split partial of every row of the block.  Returns false if a
 // pipeline wait ran out (HS2_DEV_TIMEOUT is then set).  *t_range receives the tile range.
-// Ends with the block synchronised; the ring is free again afterwards.
-template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8>
+// Ends with the block synchronised; the ring is free again afterwards.  TR (FP8, RT = 1, at most 8
+// query-head rows in the block): the transposed warp attention of attn_core_t.cuh.
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR = false>
 __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttnArgs& a,
                                            uint8_t* smem, int split, int unit, int2* t_range) {
     constexpr int NKS = NC / RT;          // warps sharing one row tile (each a key slice)
     constexpr int KW = kKeyTile / NKS;    // keys per warp per tile
     static_assert(NC % RT == 0 && KW % 16 == 0, "bad warp split");
+    static_assert(!TR || (FP8 && RT == 1 && KW == 16 && NC / RT > 1), "transposed form: FP8, one 16-key slice per warp");
     using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
     uint8_t* ring = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -156,7 +158,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     const int nt = t_end - t_begin;
     *t_range = make_int2(t_begin, t_end);
 
-    OnlineSoftmax<D, FP8> st;
+    typename std::conditional<TR, OnlineSoftmaxT<D>, OnlineSoftmax<D, FP8>>::type st;
     st.init();
     const int rt = warp % RT, ks = warp / RT;
     const int g = lane >> 2, c = lane & 3;
@@ -174,6 +176,64 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             produce_tiles<D, STAGES, 2, FP8>(tmK, tmV, ring, full, empty, abort_flag, t_begin, nt, bh, a.Hkv, a.kv,
                                              a.status, a.stream_kv != 0);
         __syncwarp();
+    } else if constexpr (TR) {
+        // query rows 0..7: lane (g, c) loads row g of Q and scores rows 2c, 2c+1
+        QTileT<D> q;
+        const int rq = row_q(g);
+        q.load(a.Q, rq >= 0 ? static_cast<int64_t>(rq) * D : -1);
+        const float f0 = a.scale_log2 * kscale * q.col_scale[0];
+        const float f1 = a.scale_log2 * kscale * q.col_scale[1];
+        const int p0 = s_pos[2 * c], p1 = s_pos[2 * c + 1];
+        const int key0 = ks * KW;
+        float* lg0 = nullptr;
+        float* lg1 = nullptr;
+        const uint64_t keep = l2_evict_last();
+        if (KEEP_LOGITS) {
+            // [row_kv][N][G]: row_kv = (b*Hkv + h)*T + t
+            if (p0 >= 0) lg0 = a.logits + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + (2 * c) / a.G) * a.N * a.G + (2 * c) % a.G;
+            if (p1 >= 0)
+                lg1 = a.logits + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + (2 * c + 1) / a.G) * a.N * a.G + (2 * c + 1) % a.G;
+        }
+        for (int i = 0; i < nt; ++i) {
+            const int stage = i % STAGES;
+            if (!mbar_wait(&full[stage], (i / STAGES) & 1, a.status)) {
+                *abort_flag = 1;
+                break;
+            }
+            if (*abort_flag) break;
+            const uint32_t kbase = smem_u32(ring + stage * L::kStageBytes);
+            const uint32_t vbase = kbase + L::kTileBytes;
+            const int tile_j0 = (t_begin + i) * kKeyTile;
+            const bool past_end = tile_j0 + key0 + KW - 1 > jmax;
+            if (past_end) {  // as below: zero this warp's V rows of keys past the CTA's last position
+                constexpr int CH = D / 16;
+                uint8_t* vtile = ring + stage * L::kStageBytes + L::kTileBytes;
+                for (int e = lane; e < KW * CH; e += 32) {
+                    const int r = key0 + e / CH;
+                    if (tile_j0 + r > jmax)
+                        *reinterpret_cast<uint4*>(vtile + kv_chunk_offset<D, FP8>(r, e % CH)) = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+            float sc[4];
+            qk_t<D>(q, kbase, key0, sc);
+            const int j_lo = tile_j0 + key0 + g, j_hi = j_lo + 8;
+            sc[0] = j_lo <= p0 ? sc[0] * f0 : -INFINITY;
+            sc[1] = j_lo <= p1 ? sc[1] * f1 : -INFINITY;
+            sc[2] = j_hi <= p0 ? sc[2] * f0 : -INFINITY;
+            sc[3] = j_hi <= p1 ? sc[3] * f1 : -INFINITY;
+            if (KEEP_LOGITS) {
+                if (j_lo <= p0) st_f32_policy(lg0 + static_cast<int64_t>(j_lo) * a.G, sc[0], keep);
+                if (j_lo <= p1) st_f32_policy(lg1 + static_cast<int64_t>(j_lo) * a.G, sc[1], keep);
+                if (j_hi <= p0) st_f32_policy(lg0 + static_cast<int64_t>(j_hi) * a.G, sc[2], keep);
+                if (j_hi <= p1) st_f32_policy(lg1 + static_cast<int64_t>(j_hi) * a.G, sc[3], keep);
+            }
+            st.update(sc, vbase, key0);
+            if (past_end) fence_async_smem();  // the zeros are ordered before the next TMA write
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+        }
+        st.finish_rows();
     } else {
         QTileOf<D, FP8> q;
         const int rq_lo = row_q(r_lo), rq_hi = row_q(r_hi);
@@ -245,11 +305,16 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
 
     const PartialRef out{a.part_ml + static_cast<int64_t>(split) * (a.B * a.Hq * a.T),
                          a.part_acc + static_cast<int64_t>(split) * (a.B * a.Hq * a.T) * D};
-    if (NKS == 1) {
+    if constexpr (NKS == 1 && !TR) {
         if (warp < NC) store_partial<D, FP8>(st, out, [&](int r) { return row_q(rt * 16 + r); }, vscale);
     } else {
         float* red = reinterpret_cast<float*>(ring);  // the ring is idle now
-        if (warp < NC) stash_state<D, NKS, FP8>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
+        if (warp < NC) {
+            if constexpr (TR)
+                stash_state_t<D, NKS>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
+            else
+                stash_state<D, NKS, FP8>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
+        }
         __syncthreads();
         // threads of the CTA split evenly over the RT tiles
         const int per = blockDim.x / RT;

@@ -103,7 +103,8 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     const int64_t units = static_cast<int64_t>(x.B) * x.Hkv * P.QB;
     if (units > 65535) return false;  // grid.y of the streaming kernels
     const int64_t tiles = (x.N + kKeyTile - 1) / kKeyTile;
-    const int64_t slots = (P.RT == 1 ? 2 : 1) * int64_t(sms);
+    // resident sweep CTAs: two per SM for 16-row blocks (three for the transposed FP8 form), else one
+    const int64_t slots = (P.RT == 1 ? (P.fp8 && x.T * G <= 8 ? 3 : 2) : 1) * int64_t(sms);
     P.S1 = choose_splits(units, tiles, slots, 256);
     P.S2 = P.S1;
     // 128-row query tiles: the full sweep runs on the tcgen05 tensor cores (HS2_UMMA=0 keeps the
@@ -136,14 +137,16 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     // kernel's combine CTA G * S1 weights in its histogram scratch
     if (static_cast<int64_t>(G) * P.S4 > 8192 || static_cast<int64_t>(G) * P.S1 > 4096) return false;
     P.cand_cap = std::min<int64_t>(x.N, std::max<int64_t>(2048, (int64_t(1) << 24) / rows_kv));
-    // one-launch decode step (HS2_FUSED_DECODE=1; it measured slower than the kernel chain at every
-    // decode shape: its row barriers and per-CTA latency chains cost more than the launches they
-    // save): one selection row per row block, kept logits, every candidate list able to hold a
-    // whole pool, a split's pool keys within the kernel's shared-memory key buffer
+    // one-launch decode step: one selection row per row block, kept logits, every candidate list
+    // able to hold a whole pool, a split's pool keys within the kernel's shared-memory key buffer.
+    // Taken for short caches, where the kernel chain is all launch and dependency latency (it
+    // measured faster at N = 2K, slower from N = 32K on: its row barriers and per-CTA latency
+    // chains then cost more than the launches they save); HS2_FUSED_DECODE=1 / 0 forces it on / off
     const char* want_fused = std::getenv("HS2_FUSED_DECODE");
     const int64_t tiles64 = (static_cast<int64_t>(x.N) + kKeyTile - 1) / kKeyTile;
-    P.fused = x.T == 1 && P.RT == 1 && P.mat_logits && !P.umma && P.cand_cap >= x.N &&
-              ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap && want_fused && want_fused[0] == '1';
+    const bool fused_ok = x.T == 1 && P.RT == 1 && P.mat_logits && !P.umma && P.cand_cap >= x.N &&
+                          ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap;
+    P.fused = fused_ok && (want_fused ? want_fused[0] == '1' : x.N <= kFusedMaxN);
     const int64_t sparse_slots = P.fused ? std::max<int64_t>(P.S4, P.S1) : P.S4;
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
     // bracketed selection (tcgen05 score sweep, many rows, large pools): a 1/16 tile sample per

@@ -29,6 +29,7 @@ enum TopkMeta { kMetaBin = 0, kMetaAbove = 1, kMetaDef = 2, kMetaCand = 3, kMeta
                 kMetaSparseDone = 6, kMetaBarrier = 7 };  // kMetaDef/kMetaCand share one 8-byte word
 constexpr int kSmemCand = 4096;      // candidates the final select keeps in shared memory
 constexpr int kFusedKeyCap = 16384;  // pool keys per split of the one-launch decode step
+constexpr int kFusedMaxN = 8192;     // the one-launch decode step by default up to this cache length
 constexpr int kMaxKW = 1 << 22;      // largest supported k + W
 constexpr int kSparseMaxC4 = 4096;         // most selected keys one sparse-attention CTA takes
 constexpr int kRowsPerCtaTopkPerSM = 4;   // from 4 x (SMs) selection rows on, one top-k CTA per row

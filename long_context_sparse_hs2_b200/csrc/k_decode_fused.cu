@@ -290,7 +290,8 @@ __global__ void __launch_bounds__(kFThreads, 2)
 
     // ---- 1. the sweep of this split: partials and kept logits
     int2 range;
-    bool ok = full_sweep<D, 1, kFNC, STAGES, true, FP8>(&tmK, &tmV, a, smem, split, row, &range);
+    constexpr bool TR = FP8 && G <= 8;  // the transposed warp attention for an FP8 cache
+    bool ok = full_sweep<D, 1, kFNC, STAGES, true, FP8, TR>(&tmK, &tmV, a, smem, split, row, &range);
     if (tid == 0) {
         uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R::kBarOff);
         for (int i = 0; i < 2 * STAGES; ++i) mbar_inval(&bars[i]);  // the memory is reused below

@@ -21,7 +21,7 @@ namespace hs2 {
 
 // ====================================================================== full attention
 
-template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8>
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR>
 __global__ void __launch_bounds__((NC + 1) * 32)
     full_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const AttnArgs a) {
@@ -35,7 +35,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             a.zero[i] = make_uint4(0, 0, 0, 0);
     }
     int2 range;
-    full_sweep<D, RT, NC, STAGES, KEEP_LOGITS, FP8>(&tmK, &tmV, a, smem, blockIdx.x, blockIdx.y, &range);
+    full_sweep<D, RT, NC, STAGES, KEEP_LOGITS, FP8, TR>(&tmK, &tmV, a, smem, blockIdx.x, blockIdx.y, &range);
     // The sweep reads nothing its predecessor writes, but it must not complete before the
     // predecessor does (later kernels rely on that chain).
     pdl_wait();
@@ -218,15 +218,19 @@ cudaError_t set_smem(Kern kern, int bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int D, int RT, bool KEEP, bool FP8>
+template <int D, int RT, bool KEEP, bool FP8, bool TR = false>
 cudaError_t full_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                               cudaStream_t st, bool pdl) {
+    // FP8 with at most 8 query-head rows per row block: the transposed warp attention
+    if constexpr (FP8 && RT == 1 && !TR)
+        if (p.T * p.G <= 8) return full_attn_variant<D, RT, KEEP, FP8, true>(p, tmK, tmV, a, st, pdl);
     constexpr int NC = RT >= 8 ? 8 : 4;
-    // ring of 96 KB (bf16: 3 stages at d = 128, 6 at d = 64; FP8 twice as many), two CTAs per SM
-    constexpr int STAGES = (D == 128 ? 3 : 6) * (FP8 ? 2 : 1);
+    // ring of 96 KB (bf16: 3 stages at d = 128, 6 at d = 64; FP8 twice as many), two CTAs per SM;
+    // the transposed FP8 form (96 registers) takes a 64 KB ring and three CTAs per SM
+    constexpr int STAGES = TR ? (D == 128 ? 4 : 8) : (D == 128 ? 3 : 6) * (FP8 ? 2 : 1);
     using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
     static_assert(L::kRingBytes >= RT * merge_floats<D, NC / RT>() * 4, "merge scratch must fit in the ring");
-    auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP, FP8>;
+    auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP, FP8, TR>;
     cudaError_t e = set_smem(kern, L::kBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S1, p.B * p.Hkv * p.QB);

@@ -242,10 +242,9 @@ TAIL_CASES = [c for c in CASES if c[5] * (c[1] // c[2]) <= 16]
 def test_decode_tail_paths_match_oracle(case, path, monkeypatch):
     # the decode tail after the sweep: the cluster tail (selection + sparse layer in one cluster
     # kernel), the kernel chain (score_hist -> topk_select -> sparse_attn), and, for T = 1, the
-    # whole step in one cooperative launch (HS2_FUSED_DECODE=1)
-    if path == "fused":
-        monkeypatch.setenv("HS2_FUSED_DECODE", "1")
-    else:
+    # whole step in one cooperative launch (HS2_FUSED_DECODE=1; the default for short caches)
+    monkeypatch.setenv("HS2_FUSED_DECODE", "1" if path == "fused" else "0")
+    if path != "fused":
         monkeypatch.setenv("HS2_CLUSTER_TAIL", "1" if path == "cluster" else "0")
     B, Hq, Hkv, d, N, T, k, W = case
     inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 7, needles=4)
