@@ -117,7 +117,7 @@ __device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, ui
 // split's K/V tiles through the TMA ring, keeps the online softmax, optionally stores the
 // base-2 logits, and writes the split partial of every row of the block.  Returns false if a
 // pipeline wait ran out (HS2_DEV_TIMEOUT is then set).  *t_range receives the tile range.
-// Ends with the block synchronised; the ring is free again afterwards.  TR (FP8, RT = 1, at most 8
+// Ends with the block synchronised; the ring is free again afterwards.  TR (RT = 1, at most 8
 // query-head rows in the block): the transposed warp attention of attn_core_t.cuh.
 template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR = false>
 __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttnArgs& a,
@@ -125,7 +125,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     constexpr int NKS = NC / RT;          // warps sharing one row tile (each a key slice)
     constexpr int KW = kKeyTile / NKS;    // keys per warp per tile
     static_assert(NC % RT == 0 && KW % 16 == 0, "bad warp split");
-    static_assert(!TR || (FP8 && RT == 1 && KW == 16 && NC / RT > 1), "transposed form: FP8, one 16-key slice per warp");
+    static_assert(!TR || (RT == 1 && KW == 16 && NC / RT > 1), "transposed form: one 16-key slice per warp");
     using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
     uint8_t* ring = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -158,7 +158,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     const int nt = t_end - t_begin;
     *t_range = make_int2(t_begin, t_end);
 
-    typename std::conditional<TR, OnlineSoftmaxT<D>, OnlineSoftmax<D, FP8>>::type st;
+    typename std::conditional<TR, OnlineSoftmaxT<D, FP8>, OnlineSoftmax<D, FP8>>::type st;
     st.init();
     const int rt = warp % RT, ks = warp / RT;
     const int g = lane >> 2, c = lane & 3;
@@ -178,7 +178,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
         __syncwarp();
     } else if constexpr (TR) {
         // query rows 0..7: lane (g, c) loads row g of Q and scores rows 2c, 2c+1
-        QTileT<D> q;
+        QTileT<D, FP8> q;
         const int rq = row_q(g);
         q.load(a.Q, rq >= 0 ? static_cast<int64_t>(rq) * D : -1);
         const float f0 = a.scale_log2 * kscale * q.col_scale[0];
@@ -206,7 +206,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             const int tile_j0 = (t_begin + i) * kKeyTile;
             const bool past_end = tile_j0 + key0 + KW - 1 > jmax;
             if (past_end) {  // as below: zero this warp's V rows of keys past the CTA's last position
-                constexpr int CH = D / 16;
+                constexpr int CH = D * (FP8 ? 1 : 2) / 16;
                 uint8_t* vtile = ring + stage * L::kStageBytes + L::kTileBytes;
                 for (int e = lane; e < KW * CH; e += 32) {
                     const int r = key0 + e / CH;
@@ -216,7 +216,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
                 __syncwarp();
             }
             float sc[4];
-            qk_t<D>(q, kbase, key0, sc);
+            qk_t<D, FP8>(q, kbase, key0, sc);
             const int j_lo = tile_j0 + key0 + g, j_hi = j_lo + 8;
             sc[0] = j_lo <= p0 ? sc[0] * f0 : -INFINITY;
             sc[1] = j_lo <= p1 ? sc[1] * f1 : -INFINITY;
@@ -311,7 +311,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
         float* red = reinterpret_cast<float*>(ring);  // the ring is idle now
         if (warp < NC) {
             if constexpr (TR)
-                stash_state_t<D, NKS>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
+                stash_state_t<D, NKS, FP8>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
             else
                 stash_state<D, NKS, FP8>(st, ks, red + rt * merge_floats<D, NKS>(), vscale);
         }

@@ -104,7 +104,9 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     if (units > 65535) return false;  // grid.y of the streaming kernels
     const int64_t tiles = (x.N + kKeyTile - 1) / kKeyTile;
     // resident sweep CTAs: two per SM for 16-row blocks (three for the transposed FP8 form), else one
-    const int64_t slots = (P.RT == 1 ? (P.fp8 && x.T * G <= 8 ? 3 : 2) : 1) * int64_t(sms);
+    const char* want_tr = std::getenv("HS2_TRANSPOSED");
+    const bool tr = x.T * G <= 8 && !(want_tr && want_tr[0] == '0');
+    const int64_t slots = (P.RT == 1 ? (P.fp8 && tr ? 3 : 2) : 1) * int64_t(sms);
     P.S1 = choose_splits(units, tiles, slots, 256);
     P.S2 = P.S1;
     // 128-row query tiles: the full sweep runs on the tcgen05 tensor cores (HS2_UMMA=0 keeps the
@@ -147,6 +149,10 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
     const bool fused_ok = x.T == 1 && P.RT == 1 && P.mat_logits && !P.umma && P.cand_cap >= x.N &&
                           ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap;
     P.fused = fused_ok && (want_fused ? want_fused[0] == '1' : x.N <= kFusedMaxN);
+    if (P.fused && P.S1 * units > 2 * int64_t(sms)) {  // the one-launch kernel holds two CTAs per SM
+        P.S1 = P.S2 = choose_splits(units, tiles, 2 * int64_t(sms), 256);
+        P.fused = ((tiles64 + P.S1 - 1) / P.S1) * kKeyTile <= kFusedKeyCap;
+    }
     const int64_t sparse_slots = P.fused ? std::max<int64_t>(P.S4, P.S1) : P.S4;
     P.kstride = ((static_cast<int64_t>(x.N) + 63) / 64) * 64;
     // bracketed selection (tcgen05 score sweep, many rows, large pools): a 1/16 tile sample per

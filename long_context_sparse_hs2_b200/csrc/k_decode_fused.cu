@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kFThreads, 2)
 
     // ---- 1. the sweep of this split: partials and kept logits
     int2 range;
-    constexpr bool TR = FP8 && G <= 8;  // the transposed warp attention for an FP8 cache
+    constexpr bool TR = G <= 8;  // the transposed warp attention (at most 8 query-head rows)
     bool ok = full_sweep<D, 1, kFNC, STAGES, true, FP8, TR>(&tmK, &tmV, a, smem, split, row, &range);
     if (tid == 0) {
         uint64_t* bars = reinterpret_cast<uint64_t*>(smem + R::kBarOff);

@@ -11,6 +11,7 @@
 // combine_kernel: split partials -> bf16 O and natural-log LSE (used when the combine is not
 // fused into the next kernel).
 #include <algorithm>
+#include <cstdlib>
 
 #include "attn_sweep.cuh"
 #include "combine.cuh"
@@ -213,6 +214,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 
 namespace {
 
+// HS2_TRANSPOSED=0 keeps the query-rows-as-M warp attention for decode row blocks
+bool transposed_decode() {
+    const char* env = std::getenv("HS2_TRANSPOSED");
+    return !(env && env[0] == '0');
+}
+
 template <class Kern>
 cudaError_t set_smem(Kern kern, int bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -221,13 +228,13 @@ cudaError_t set_smem(Kern kern, int bytes) {
 template <int D, int RT, bool KEEP, bool FP8, bool TR = false>
 cudaError_t full_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                               cudaStream_t st, bool pdl) {
-    // FP8 with at most 8 query-head rows per row block: the transposed warp attention
-    if constexpr (FP8 && RT == 1 && !TR)
-        if (p.T * p.G <= 8) return full_attn_variant<D, RT, KEEP, FP8, true>(p, tmK, tmV, a, st, pdl);
+    // at most 8 query-head rows per row block: the transposed warp attention
+    if constexpr (RT == 1 && !TR)
+        if (p.T * p.G <= 8 && transposed_decode()) return full_attn_variant<D, RT, KEEP, FP8, true>(p, tmK, tmV, a, st, pdl);
     constexpr int NC = RT >= 8 ? 8 : 4;
     // ring of 96 KB (bf16: 3 stages at d = 128, 6 at d = 64; FP8 twice as many), two CTAs per SM;
     // the transposed FP8 form (96 registers) takes a 64 KB ring and three CTAs per SM
-    constexpr int STAGES = TR ? (D == 128 ? 4 : 8) : (D == 128 ? 3 : 6) * (FP8 ? 2 : 1);
+    constexpr int STAGES = (TR && FP8) ? (D == 128 ? 4 : 8) : (D == 128 ? 3 : 6) * (FP8 ? 2 : 1);
     using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
     static_assert(L::kRingBytes >= RT * merge_floats<D, NC / RT>() * 4, "merge scratch must fit in the ring");
     auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP, FP8, TR>;
