@@ -40,7 +40,8 @@ struct StreamSmem {
     static constexpr int kRingBytes = STAGES * kStageBytes;
     static constexpr int kBarOff = kRingBytes;                           // full[STAGES], empty[STAGES]
     static constexpr int kMiscOff = kBarOff + 2 * STAGES * 8;            // abort flag + row positions
-    static constexpr int kBytes = kMiscOff + 16 + 128 * 4 + 1024;        // + alignment slack
+    static constexpr int kTileOff = kMiscOff + 16 + 128 * 4;           // key tile of each stage (dynamic sweep)
+    static constexpr int kBytes = kTileOff + 16 * 4 + 1024;              // + alignment slack
 };
 
 // Issues the TMA loads of one tile (keys j0 .. j0 + 63 of kv slice bh = b*Hkv + h) of one tensor
@@ -113,13 +114,70 @@ __device__ void produce_tiles(const CUtensorMap* tmK, const CUtensorMap* tmV, ui
 }
 
 
+// Producer side of the dynamically scheduled sweep: the CTAs of a row block take chunks of
+// `chunk` consecutive key tiles of [0, ntiles) from the counter ctr (one atomic per chunk, the next
+// chunk taken while the current one is loading), so that a CTA that finishes early takes more
+// and all of them end together.  The tile of each stage goes to s_tile[stage] before its loads;
+// a final stage with no loads and tile -1 tells the consumers to stop.
+template <int D, int STAGES, bool FP8>
+__device__ void produce_tiles_dyn(const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* ring, uint64_t* full,
+                                  uint64_t* empty, volatile int* abort_flag, int* s_tile, int* ctr, int ntiles,
+                                  int chunk, int bh, int Hkv, const KvSrc& kv, unsigned* status, bool stream) {
+    using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
+    const uint64_t pol = stream ? l2_evict_first() : l2_evict_normal();
+    prefetch_tensormap(tmK);
+    prefetch_tensormap(tmV);
+    int i = 0, issued = 0;
+    bool ok = true;
+    pdl_wait();  // the counter is cleared by the call's first kernel
+    int cur = atomicAdd(ctr, chunk);
+    // (the counter only grows from 0, so a CTA never takes more than ntiles tiles; the bound on
+    // issued makes that explicit)
+    while (ok && cur >= 0 && cur < ntiles && issued < ntiles) {
+        const int nxt = atomicAdd(ctr, chunk);
+        const int end = min(cur + chunk, ntiles);
+        for (int t = cur; t < end; ++t, ++i) {
+            const int stage = i % STAGES;
+            if ((i >= STAGES && !mbar_wait(&empty[stage], ((i / STAGES) - 1) & 1, status)) || *abort_flag) {
+                *abort_flag = 1;
+                ok = false;
+                break;
+            }
+            s_tile[stage] = t;
+            mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+            uint8_t* dst = ring + stage * L::kStageBytes;
+            load_kv_tile<D, FP8>(dst, tmK, &full[stage], kv, t * kKeyTile, bh, Hkv, pol, status);
+            load_kv_tile<D, FP8>(dst + L::kTileBytes, tmV, &full[stage], kv, t * kKeyTile, bh, Hkv, pol, status);
+            ++issued;
+        }
+        cur = nxt;
+    }
+    // drain: the last load issued into every stage has landed before the CTA retires (done before
+    // the end marker, whose plain arrive completes one more phase of its stage's barrier)
+    for (int st = 0; st < STAGES && st < issued; ++st) {
+        const int last = st + ((issued - 1 - st) / STAGES) * STAGES;
+        mbar_wait(&full[st], (last / STAGES) & 1, status);
+    }
+    if (ok) {  // the end marker
+        const int stage = i % STAGES;
+        if (i < STAGES || mbar_wait(&empty[stage], ((i / STAGES) - 1) & 1, status)) {
+            s_tile[stage] = -1;
+            mbar_arrive(&full[stage]);
+        } else {
+            *abort_flag = 1;
+        }
+    }
+}
+
 // One CTA's share of the full-attention sweep: row block `unit`, split `split`.  Streams the
 // split's K/V tiles through the TMA ring, keeps the online softmax, optionally stores the
 // base-2 logits, and writes the split partial of every row of the block.  Returns false if a
 // pipeline wait ran out (HS2_DEV_TIMEOUT is then set).  *t_range receives the tile range.
 // Ends with the block synchronised; the ring is free again afterwards.  TR (RT = 1, at most 8
-// query-head rows in the block): the transposed warp attention of attn_core_t.cuh.
-template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR = false>
+// query-head rows in the block): the transposed warp attention of attn_core_t.cuh.  DYN: the
+// split's tiles are not a fixed range but chunks taken from a.tilectr[unit] (produce_tiles_dyn);
+// *t_range is then empty.
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR = false, bool DYN = false>
 __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtensorMap* tmV, const AttnArgs& a,
                                            uint8_t* smem, int split, int unit, int2* t_range) {
     constexpr int NKS = NC / RT;          // warps sharing one row tile (each a key slice)
@@ -156,7 +214,10 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     const int t_begin = static_cast<int>((static_cast<int64_t>(split) * ntiles) / a.S);
     const int t_end = static_cast<int>((static_cast<int64_t>(split + 1) * ntiles) / a.S);
     const int nt = t_end - t_begin;
-    *t_range = make_int2(t_begin, t_end);
+    *t_range = DYN ? make_int2(0, 0) : make_int2(t_begin, t_end);
+    int* s_tile = reinterpret_cast<int*>(smem + L::kTileOff);
+    // the key tile of step i: fixed range, or what the producer put in the stage (-1: the end)
+    auto tile_of = [&](int i, int stage) -> int { return DYN ? s_tile[stage] : t_begin + i; };
 
     typename std::conditional<TR, OnlineSoftmaxT<D, FP8>, OnlineSoftmax<D, FP8>>::type st;
     st.init();
@@ -172,9 +233,15 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
     const float kscale = FP8 ? a.kv.k_scale[bh] : 1.f;
     const float vscale = FP8 ? a.kv.v_scale[bh] : 1.f;
     if (warp == NC) {
-        if (lane == 0)
-            produce_tiles<D, STAGES, 2, FP8>(tmK, tmV, ring, full, empty, abort_flag, t_begin, nt, bh, a.Hkv, a.kv,
-                                             a.status, a.stream_kv != 0);
+        if (lane == 0) {
+            if (DYN)
+                produce_tiles_dyn<D, STAGES, FP8>(tmK, tmV, ring, full, empty, abort_flag, s_tile, a.tilectr + unit,
+                                                  ntiles, max(1, ntiles / (a.S * 8)), bh, a.Hkv, a.kv, a.status,
+                                                  a.stream_kv != 0);
+            else
+                produce_tiles<D, STAGES, 2, FP8>(tmK, tmV, ring, full, empty, abort_flag, t_begin, nt, bh, a.Hkv,
+                                                 a.kv, a.status, a.stream_kv != 0);
+        }
         __syncwarp();
     } else if constexpr (TR) {
         // query rows 0..7: lane (g, c) loads row g of Q and scores rows 2c, 2c+1
@@ -194,7 +261,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             if (p1 >= 0)
                 lg1 = a.logits + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + (2 * c + 1) / a.G) * a.N * a.G + (2 * c + 1) % a.G;
         }
-        for (int i = 0; i < nt; ++i) {
+        for (int i = 0; DYN || i < nt; ++i) {
             const int stage = i % STAGES;
             if (!mbar_wait(&full[stage], (i / STAGES) & 1, a.status)) {
                 *abort_flag = 1;
@@ -203,7 +270,9 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             if (*abort_flag) break;
             const uint32_t kbase = smem_u32(ring + stage * L::kStageBytes);
             const uint32_t vbase = kbase + L::kTileBytes;
-            const int tile_j0 = (t_begin + i) * kKeyTile;
+            const int tile = tile_of(i, stage);
+            if (tile < 0) break;  // the end marker of the dynamic sweep
+            const int tile_j0 = tile * kKeyTile;
             const bool past_end = tile_j0 + key0 + KW - 1 > jmax;
             if (past_end) {  // as below: zero this warp's V rows of keys past the CTA's last position
                 constexpr int CH = D * (FP8 ? 1 : 2) / 16;
@@ -252,7 +321,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             if (p_hi >= 0)
                 lg_hi = a.logits + (static_cast<int64_t>(bh) * a.T + qb * a.TQ + r_hi / a.G) * a.N * a.G + (r_hi % a.G);
         }
-        for (int i = 0; i < nt; ++i) {
+        for (int i = 0; DYN || i < nt; ++i) {
             const int stage = i % STAGES;
             if (!mbar_wait(&full[stage], (i / STAGES) & 1, a.status)) {
                 *abort_flag = 1;
@@ -261,7 +330,9 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             if (*abort_flag) break;
             const uint32_t kbase = smem_u32(ring + stage * L::kStageBytes);
             const uint32_t vbase = kbase + L::kTileBytes;
-            const int tile_j0 = (t_begin + i) * kKeyTile;
+            const int tile = tile_of(i, stage);
+            if (tile < 0) break;  // the end marker of the dynamic sweep
+            const int tile_j0 = tile * kKeyTile;
             const bool past_end = tile_j0 + key0 + KW - 1 > jmax;
             if (past_end) {
                 // Keys past the CTA's last position are masked (P = 0), but their cache slots may hold
@@ -278,7 +349,7 @@ __device__ __forceinline__ bool full_sweep(const CUtensorMap* tmK, const CUtenso
             }
             float sc[KW / 8][4];
             qk_any<D, KW, FP8>(q, kbase, key0, sc);
-            const int jb = (t_begin + i) * kKeyTile + key0 + 2 * c;
+            const int jb = tile_j0 + key0 + 2 * c;
 #pragma unroll
             for (int n = 0; n < KW / 8; ++n) {
 #pragma unroll

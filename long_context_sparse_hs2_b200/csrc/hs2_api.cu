@@ -174,6 +174,8 @@ bool make_plan(const hs2_dims* dm, Plan* p, hs2_status* why, const KvShape& kv) 
 
     size_t off = 0;
     P.off_status = off; off += 256;
+    P.off_tilectr = off; off = align_up(off + size_t(units) * 4, 256);  // cleared by every call's init
+    P.init_bytes = off;
     P.off_pos = off; off = align_up(off + size_t(x.B) * 4, 256);  // decode step: the positions it runs at
     P.off_meta = off; off = align_up(off + rows_kv * kMetaInts * 4, 256);
     P.meta_end = off;
@@ -288,6 +290,7 @@ AttnArgs attn_args(const Plan& p, const void* Q, const int32_t* pos, const KvVie
     a.part_acc = w.at<float>(p.off_pf_acc);
     a.kv = kv.src;
     a.status = w.at<unsigned>(p.off_status);
+    a.tilectr = w.at<int>(p.off_tilectr);
     return a;
 }
 
@@ -575,7 +578,7 @@ hs2_status full_attn_impl(const Plan& p, const KvView& kv, const void* Q_full, c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(launch_init(ws, 256, st));
+    HS2_TRY(launch_init(ws, p.init_bytes, st));  // status word and the sweep's tile counters
     return run_full(p, Q_full, kv, pos, O_full, LSE_full, w, false, true, 0, 0, st);
 }
 
@@ -619,9 +622,9 @@ hs2_status step_impl(const Plan& p, const KvView& kv, const void* Q_full, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    // status word (and, for the one-launch decode step, the counters and histograms; otherwise
-    // the full sweep clears those for the kernels after it)
-    HS2_TRY(launch_init(ws, p.fused ? p.zero_bytes : 256, st));
+    // status word and the sweep's tile counters (and, for the one-launch decode step, the per-row
+    // counters and histograms; otherwise the full sweep clears those for the kernels after it)
+    HS2_TRY(launch_init(ws, p.fused ? p.zero_bytes : p.init_bytes, st));
     return run_step(p, Q_full, Q_sparse, kv, pos, O_full, O_sparse, LSE_full, LSE_sparse, idx, cnt, w, st, true);
 }
 
@@ -771,7 +774,7 @@ hs2_status hs2_decode_step(const hs2_dims* dims, const hs2_kv_cache* cache, cons
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Ws w{static_cast<uint8_t*>(ws)};
     trace_call_begin(st);
-    HS2_TRY(launch_init(ws, p.fused ? p.zero_bytes : 256, st));  // status word (+ counters: see step_impl)
+    HS2_TRY(launch_init(ws, p.fused ? p.zero_bytes : p.init_bytes, st));  // as in step_impl
     // the new tokens go in and pos advances; the step then reads the positions from ws.  The full
     // sweep is an ordinary launch, so it starts after the append has completed and every kernel
     // after it sees the new tokens and positions.

@@ -85,7 +85,7 @@ struct Plan {
     int64_t sstride;    // sample keys per row (a multiple of 128)
     int64_t bcap;       // candidate-list capacity per row
     // workspace byte offsets
-    size_t off_status, off_pos, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand, off_segcnt,
+    size_t off_status, off_tilectr, init_bytes, off_pos, off_meta, meta_end, off_hist, off_pf_ml, off_pf_acc, off_ps_ml, off_ps_acc, off_keys, off_cand, off_segcnt,
         off_logits, zero_bytes, total;
 };
 
@@ -110,6 +110,8 @@ struct AttnArgs {
     int TQ, QB, S;
     float scale_log2;      // d^-1/2 * log2(e)
     int stream_kv;         // 1: every K/V tile is read once (decode) -> load it evict-first
+    int* tilectr;          // [units] tiles handed out so far (the mma.sync full sweep's CTAs of a row
+                           // block take chunks of its key tiles from it); cleared by init
     float2* part_ml;       // [S][rows_q]
     float* part_acc;       // [S][rows_q][D]
     float* logits;         // optional [rows_kv][N][G] base-2 logits (full sweep only)

@@ -22,7 +22,7 @@ namespace hs2 {
 
 // ====================================================================== full attention
 
-template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR>
+template <int D, int RT, int NC, int STAGES, bool KEEP_LOGITS, bool FP8, bool TR, bool DYN>
 __global__ void __launch_bounds__((NC + 1) * 32)
     full_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const AttnArgs a) {
@@ -36,7 +36,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
             a.zero[i] = make_uint4(0, 0, 0, 0);
     }
     int2 range;
-    full_sweep<D, RT, NC, STAGES, KEEP_LOGITS, FP8, TR>(&tmK, &tmV, a, smem, blockIdx.x, blockIdx.y, &range);
+    full_sweep<D, RT, NC, STAGES, KEEP_LOGITS, FP8, TR, DYN>(&tmK, &tmV, a, smem, blockIdx.x, blockIdx.y, &range);
     // The sweep reads nothing its predecessor writes, but it must not complete before the
     // predecessor does (later kernels rely on that chain).
     pdl_wait();
@@ -214,6 +214,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 
 namespace {
 
+constexpr int64_t kDynMinTiles = 128;  // key tiles per CTA from which the sweep is scheduled dynamically
+
 // HS2_TRANSPOSED=0 keeps the query-rows-as-M warp attention for decode row blocks
 bool transposed_decode() {
     const char* env = std::getenv("HS2_TRANSPOSED");
@@ -225,19 +227,32 @@ cudaError_t set_smem(Kern kern, int bytes) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int D, int RT, bool KEEP, bool FP8, bool TR = false>
+template <int D, int RT, bool KEEP, bool FP8, bool TR = false, int DYN = -1>
 cudaError_t full_attn_variant(const Plan& p, const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnArgs& a,
                               cudaStream_t st, bool pdl) {
+    // Long key ranges per CTA (at least kDynMinTiles tiles: the 1M-token decode) are handed out in
+    // chunks from a counter, so that CTAs slowed by memory contention take fewer of them (4-5 %
+    // faster there); shorter ranges keep a fixed split (the counter cost more than it saved at
+    // the 32K-token batch and broke even at 128K), which also keeps their summation order fixed.
+    // HS2_DYN_SWEEP=1 / 0 forces either.
+    if constexpr (DYN < 0) {
+        const char* env = std::getenv("HS2_DYN_SWEEP");
+        const int64_t tiles = (static_cast<int64_t>(p.N) + kKeyTile - 1) / kKeyTile;
+        const bool dyn = env ? env[0] == '1' : (tiles + p.S1 - 1) / p.S1 >= kDynMinTiles;
+        return dyn ? full_attn_variant<D, RT, KEEP, FP8, TR, 1>(p, tmK, tmV, a, st, pdl)
+                   : full_attn_variant<D, RT, KEEP, FP8, TR, 0>(p, tmK, tmV, a, st, pdl);
+    }
     // at most 8 query-head rows per row block: the transposed warp attention
     if constexpr (RT == 1 && !TR)
-        if (p.T * p.G <= 8 && transposed_decode()) return full_attn_variant<D, RT, KEEP, FP8, true>(p, tmK, tmV, a, st, pdl);
+        if (p.T * p.G <= 8 && transposed_decode())
+            return full_attn_variant<D, RT, KEEP, FP8, true, DYN>(p, tmK, tmV, a, st, pdl);
     constexpr int NC = RT >= 8 ? 8 : 4;
     // ring of 96 KB (bf16: 3 stages at d = 128, 6 at d = 64; FP8 twice as many), two CTAs per SM;
     // the transposed FP8 form (96 registers) takes a 64 KB ring and three CTAs per SM
     constexpr int STAGES = (TR && FP8) ? (D == 128 ? 4 : 8) : (D == 128 ? 3 : 6) * (FP8 ? 2 : 1);
     using L = StreamSmem<D, STAGES, 2, FP8 ? 1 : 2>;
     static_assert(L::kRingBytes >= RT * merge_floats<D, NC / RT>() * 4, "merge scratch must fit in the ring");
-    auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP, FP8, TR>;
+    auto kern = full_attn_kernel<D, RT, NC, STAGES, KEEP, FP8, TR, (DYN == 1)>;
     cudaError_t e = set_smem(kern, L::kBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S1, p.B * p.Hkv * p.QB);

@@ -92,6 +92,20 @@ def test_step_matches_oracle(case):
     compare_step(inp, res)
 
 
+DYN_CASES = [c for c in CASES if c[5] * (c[1] // c[2]) <= 64][:5]
+
+
+@pytest.mark.parametrize("case", DYN_CASES, ids=[str(c) for c in DYN_CASES])
+def test_step_with_dynamically_scheduled_sweep(case, monkeypatch):
+    # the full sweep's CTAs taking their key tiles in chunks from a per-row-block counter (the
+    # default only for very long caches) must give the same results
+    monkeypatch.setenv("HS2_DYN_SWEEP", "1")
+    monkeypatch.setenv("HS2_FUSED_DECODE", "0")
+    B, Hq, Hkv, d, N, T, k, W = case
+    inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 3, needles=4)
+    compare_step(inp, run_step(inp))
+
+
 def test_positions_before_the_window_and_first_token():
     # pos < W (empty pool), pos = 0 (one visible key), and arbitrary positions per batch row
     pos = np.array([[0, 3, 10, 700], [5, 64, 65, 999]], np.int32)
