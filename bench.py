@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn queries/s and achieved HBM GB/s (% of 8 TB/s) at N=128K, 1xB200"
 # DRAM bytes (read + write) per launch of the roofline kernel, from an ncu capture of the same
 # kernel binary on the same workload; None where no capture matches the current kernel.
-NCU_TRAFFIC = {("long", "full_attn_keep_logits"): 536951296 + 6840320}
+NCU_TRAFFIC = {("long", "full_attn_keep_logits"): 536944384 + 8409600}
 NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1000 * 1000
 L2_FLUSH_BYTES = 256 << 20

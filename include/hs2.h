@@ -133,13 +133,16 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, c
  * stream, sharing intermediates through ws.  When T*G <= 16 the full-attention pass keeps its
  * logits so the selection does not read K a second time; when T*G > 64 (128-row query tiles:
  * chunked prefill, multi-query decode) the full-attention and score sweeps run on the tcgen05
- * tensor cores.  Two environment variables change the execution plan (results are the same up
- * to rounding order; the workspace size depends on them, so query hs2_workspace_size under the
- * same environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles, and
- * HS2_CLUSTER_TAIL=1 / 0 forces the decode tail after the sweep (T*G <= 16) onto one
- * thread-block cluster per selection row / onto the three-kernel chain (by default each shape
- * takes the one measured faster for it).  The plan, and so the workspace size, also follows the
- * current device's SM count. */
+ * tensor cores.  Environment variables change the execution plan (results are the same up to
+ * rounding order; the workspace size depends on them, so query hs2_workspace_size under the same
+ * environment): HS2_UMMA=0 keeps the warp-level MMA sweeps for 128-row tiles;
+ * HS2_PREFILL_BRACKET=0 stores every selection key for many rows over long caches instead of
+ * filtering candidates; HS2_TRANSPOSED=0 keeps the 16-row warp attention for decode row blocks;
+ * HS2_DYN_SWEEP=1 / 0 forces the counter-scheduled sweep on / off (default: on for at least 128
+ * key tiles per CTA); HS2_FUSED_DECODE=1 / 0 forces the one-launch decode step (T = 1) on / off
+ * (default: caches of at most 8192 tokens); HS2_CLUSTER_TAIL=1 runs the decode tail after the
+ * sweep (T*G <= 16) as one thread-block cluster per selection row instead of the three-kernel
+ * chain.  The plan, and so the workspace size, also follows the current device's SM count. */
 HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
                     const void* K, const void* V, const int32_t* pos,
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,

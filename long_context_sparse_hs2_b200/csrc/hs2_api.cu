@@ -440,10 +440,10 @@ hs2_status run_tail(const Plan& p, const void* Qs, const KvView& kv, const int32
                     void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt, const Ws& w,
                     cudaStream_t st, bool* done) {
     *done = false;
-    // HS2_CLUSTER_TAIL=0: always the kernel chain; =1: the cluster kernel wherever it fits; unset:
-    // the cluster kernel where it measured faster (see launch_tail)
+    // HS2_CLUSTER_TAIL=1: the cluster kernel wherever it fits; otherwise the kernel chain, which
+    // measured faster at every decode shape (see launch_tail)
     const char* env = std::getenv("HS2_CLUSTER_TAIL");
-    if (env && env[0] == '0') return HS2_OK;
+    if (!env || env[0] != '1') return HS2_OK;
     const bool force = env && env[0] == '1';
     TailArgs t{};
     t.logits = w.at<float>(p.off_logits);

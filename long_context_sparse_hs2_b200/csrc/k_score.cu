@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256) score_hist_kernel(const ScoreArgs a) {
     const float* lg = a.logits + row * static_cast<int64_t>(a.N) * G;
     uint32_t* keys = a.keys + row * a.kstride;
     bool nonfinite = false;
-    constexpr int U = 4;  // keys in flight per thread
+    constexpr int U = G >= 16 ? 4 : 8;  // keys in flight per thread
     for (int base = j0 + threadIdx.x; base < j1; base += U * 256) {
         float v[U][G];
 #pragma unroll

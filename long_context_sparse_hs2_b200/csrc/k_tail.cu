@@ -578,11 +578,12 @@ cudaError_t choose_tail(const Plan& p, Kern kern, bool force, TailChoice* out) {
         }
         if (static_cast<int64_t>(active) < p.rows_kv && C > 1) continue;  // not one wave: try smaller clusters
         if (active < 1) return cudaSuccess;                               // cannot run: keep the kernel chain
-        // Measured on B200: the cluster tail beats the kernel chain when its grid covers most SMs
-        // (batched decode, 32 rows x 4 CTAs: 0.1425 against 0.1459 ms) and loses slightly when it
-        // leaves them idle (long-context decode, 8 rows x 10 CTAs: 0.1306 against 0.1292 ms).
-        // Unless forced, it takes the shape only when rows x C >= 4/5 of the SMs.
-        if (!force && static_cast<int64_t>(C) * p.rows_kv * 5 < static_cast<int64_t>(p.sms) * 4) return cudaSuccess;
+        // Measured on B200: the cluster tail once beat the kernel chain where its grid covered most
+        // SMs (batched decode, 32 rows x 4 CTAs: 0.1425 against 0.1459 ms) and lost where it left
+        // them idle (long-context decode, 8 rows x 10 CTAs: 0.1306 against 0.1292 ms); since the
+        // chain's scoring and final selection were sped up it loses there too (0.1421 against
+        // 0.1381 ms), so it runs only when forced.
+        if (!force) return cudaSuccess;
         *out = TailChoice{C, s, bytes};
         return cudaSuccess;
     }

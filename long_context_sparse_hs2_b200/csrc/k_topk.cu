@@ -59,6 +59,8 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(const TopkArgs a) {
 
 // ====================================================================== select: emit, then exact threshold
 
+constexpr int kRankCand = 1024;  // up to this many threshold-bucket candidates are ranked directly
+
 __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
     __shared__ unsigned long long s_cand[kSmemCand];
     __shared__ unsigned h[256];
@@ -168,8 +170,19 @@ __global__ void __launch_bounds__(256, 3) topk_select_kernel(const TopkArgs a) {
         if (ncand <= kSmemCand) {
             for (int i = threadIdx.x; i < ncand; i += blockDim.x) s_cand[i] = __ldcg(gc + i);
             __syncthreads();
-            const SmemSource src{s_cand, ncand};
-            emit_at_least(src, radix_threshold(src, need, h, s_small), need, tail, &s_count);
+            if (ncand <= kRankCand) {
+                // few candidates: each one's rank among them (composites are distinct) is its slot,
+                // and it is selected iff that rank is below need -- one pass, no radix passes
+                for (int i = threadIdx.x; i < ncand; i += blockDim.x) {
+                    const unsigned long long c = s_cand[i];
+                    unsigned r = 0;
+                    for (int j = 0; j < ncand; ++j) r += s_cand[j] > c;
+                    if (r < need) tail[r] = composite_index(c);
+                }
+            } else {
+                const SmemSource src{s_cand, ncand};
+                emit_at_least(src, radix_threshold(src, need, h, s_small), need, tail, &s_count);
+            }
         } else {
             const GlobalSource src{gc, ncand};
             emit_at_least(src, radix_threshold(src, need, h, s_small), need, tail, &s_count);
