@@ -45,7 +45,7 @@ constexpr int kFNC = 4;                    // consumer warps (four 16-key slices
 constexpr int kFWarps = kFNC + 1;          // + the TMA producer of the sweep
 constexpr int kFThreads = kFWarps * 32;
 constexpr int kFKeyCap = kFusedKeyCap;     // pool keys of one split kept in shared memory
-constexpr int kFCandCap = 2048;            // a row's candidates ranked from shared memory
+constexpr int kFCandCap = 2048;            // a row's candidates radix-selected from shared memory
 constexpr int kFOwnCap = 1024;             // a CTA's own candidates kept in shared memory
 
 template <int D, int STAGES, bool FP8>
@@ -99,34 +99,6 @@ __device__ __forceinline__ bool row_barrier(int* ctr, int target, unsigned* stat
     }
     __syncthreads();
     return *s_flag != 0;
-}
-
-// Warp 0: the bucket b1 holding the need-th best key of histogram h (shared memory) and the
-// number of keys in better buckets, into *s_bin, *s_above.
-__device__ __forceinline__ void warp_bucket_at(const unsigned* h, unsigned need, int* s_bin, int* s_above) {
-    constexpr int PER = kHistBins / 32;
-    const int lane = threadIdx.x & 31;
-    unsigned sum = 0;
-    for (int i = 0; i < PER; ++i) sum += h[lane * PER + i];
-    unsigned incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    const unsigned excl = incl - sum;
-    if (excl < need && need <= incl) {
-        unsigned cum = excl;
-        for (int i = 0; i < PER; ++i) {
-            const unsigned v = h[lane * PER + i];
-            if (cum + v >= need) {
-                *s_bin = lane * PER + i;
-                *s_above = static_cast<int>(cum);
-                break;
-            }
-            cum += v;
-        }
-    }
 }
 
 // Exclusive prefix of v over the block and the block total (blockDim.x a multiple of 32).
