@@ -74,6 +74,18 @@ def test_workspace_follows_the_execution_plan(L, monkeypatch):
             assert hs2.workspace_size(_dims(Hq=G, Hkv=1, T=max(1, 200 // G), N=5000, d=d)) > 0, (G, d)
 
 
+def test_prefill_selection_does_not_store_every_score_key(L, monkeypatch):
+    # chunked prefill (16384 selection rows over a 128K cache): the bracketed selection keeps a
+    # 1/16 sample and candidate lists, well under 2 GB of workspace; storing every score key
+    # (HS2_PREFILL_BRACKET=0) needs the 8.6 GB key matrix
+    prefill = _dims(Hq=32, Hkv=4, T=4096, N=131072, k=2048, W=128)
+    monkeypatch.delenv("HS2_PREFILL_BRACKET", raising=False)
+    bracketed = hs2.workspace_size(prefill)
+    monkeypatch.setenv("HS2_PREFILL_BRACKET", "0")
+    stored = hs2.workspace_size(prefill)
+    assert 0 < bracketed < 2e9 and stored > 8.5e9, (bracketed, stored)
+
+
 FAKE = 1 << 20  # a 256-byte-aligned non-null address; never dereferenced (checks fail first)
 
 
