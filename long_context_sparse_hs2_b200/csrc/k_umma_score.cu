@@ -312,6 +312,16 @@ __global__ void __launch_bounds__(kSThreads, 1)
             for (int i = lane; i < nqw; i += 32) s_cnt[i] = 0;
             __syncwarp();
         }
+        // filter mode, G >= 8: the warp's query bounds in registers (the same for every tile)
+        constexpr bool kRegThr = G >= 8;
+        float qthr[2][32 / G];
+#pragma unroll
+        for (int cq = 0; cq < 2; ++cq)
+#pragma unroll
+            for (int qq = 0; qq < 32 / G; ++qq) {
+                const int ql = (32 * cq) / G + qq;
+                qthr[cq][qq] = (kRegThr && mode == 2 && ql < nqw) ? s_thr[qa0 + ql] : INFINITY;
+            }
         for (int i = 0; i < nt; ++i) {
             const int buf = i & 1;
             const bool got = mbar_wait(&sfull[buf], (i >> 1) & 1, a.status);
@@ -353,7 +363,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
                     for (int qq = 0; qq < 32 / G; ++qq) {
                         const int ql = (32 * cq) / G + qq;  // query of the warpgroup
-                        const bool take = sv[qq] > s_thr[qa0 + ql] && (fast || j <= s_pl[qa0 + ql]);
+                        const float thr = kRegThr ? qthr[cq][qq] : s_thr[qa0 + ql];
+                        const bool take = sv[qq] > thr && (fast || j <= s_pl[qa0 + ql]);
                         const unsigned bal = __ballot_sync(0xffffffffu, take);
                         if (bal == 0u) continue;
                         const int c0 = kRegCnt ? qcnt[cq][qq] : s_cnt[ql];
