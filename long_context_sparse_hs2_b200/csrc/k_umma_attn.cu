@@ -255,7 +255,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
                 for (int s = 0; ok && s < 2; ++s) {
                     const int ns = s == 0 ? nstep0 : nstep1;
                     if (i >= ns) continue;
-                    ok = !*abort_flag && issue_pv(s, i);
+                    // (no abort-flag check here: every wait below is bounded, so an aborted CTA
+                    // still ends; the flag's shared-memory load sat on the issue path)
+                    ok = issue_pv(s, i);
                     if (ok && i + 1 < ns) ok = issue_qk(s, i + 1);
                 }
             }
