@@ -17,6 +17,7 @@
 // row's last CTA to finish (a completion counter; nothing waits) merges the S4 split
 // partials into O_sparse and LSE_sparse.
 #include <algorithm>
+#include <cstdlib>
 
 #include "combine.cuh"
 #include "hs2_internal.h"
@@ -44,14 +45,16 @@ __device__ __forceinline__ void finish_row(const SparseArgs& a, int row, int64_t
     const int64_t rows_q = static_cast<int64_t>(a.B) * a.Hq * a.T;
     float* s_w = reinterpret_cast<float*>(smem);                       // G * S4 weights
     float2* s_ml = reinterpret_cast<float2*>(smem) + a.G * a.S4 / 2 + 1;  // after the weights
-    block_combine_rows<D>(a.part_ml, a.part_acc, a.S4, rows_q, rq_base, a.T, a.G, s_w, s_ml, a.O, a.LSE);
+    block_combine_rows<D, 16>(a.part_ml, a.part_acc, a.S4, rows_q, rq_base, a.T, a.G, s_w, s_ml, a.O, a.LSE);
 }
 
 }  // namespace
 
 // MINB: CTAs per SM the register allocation must allow (2 for one-step CTAs, whose ring is a
 // single 64 KB stage; 1 for the deep-ring variant, which also gets the registers to avoid spills).
-template <int D, int MINB, bool FP8>
+// TR: at most 8 query heads per kv head -- the transposed warp attention of attn_core_t.cuh
+// (keys as the MMA's M dimension, no padded rows).
+template <int D, int MINB, bool FP8, bool TR>
 __global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const SparseArgs a) {
     using L = SparseSmem<D, FP8>;
     constexpr int KW = 16;  // keys per warp per step: warps 0-3 take sub-tile 0, warps 4-7 sub-tile 1
@@ -123,53 +126,86 @@ __global__ void __launch_bounds__(kSparseThreads, MINB) sparse_attn_kernel(const
     }
 
     const int g = lane >> 2, c = lane & 3;
-    QTileOf<D, FP8> q;
-    {
-        const int r0 = row_q(g), r1 = row_q(g + 8);
-        q.load(a.Q, r0 >= 0 ? static_cast<int64_t>(r0) * D : -1, r1 >= 0 ? static_cast<int64_t>(r1) * D : -1);
-    }
     const float kscale = FP8 ? a.kv.k_scale[bh] : 1.f;
     const float vscale = FP8 ? a.kv.v_scale[bh] : 1.f;
-    const float f_lo = logit_factor<D, FP8>(q, 0, a.scale_log2, kscale);
-    const float f_hi = logit_factor<D, FP8>(q, 1, a.scale_log2, kscale);
-    OnlineSoftmax<D, FP8> st;
-    st.init();
     const int sub = warp >> 2;
     const int key0 = (warp & 3) * KW;
-    for (int i = 0; i < ntl; ++i) {
-        cp_async_wait_upto(min(ntl, i + stages) - (i + 1));  // step i has landed
-        __syncthreads();
-        const int stage = i % stages;
-        const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes + sub * L::kSubBytes);
-        const uint32_t vbase = kbase + L::kTileBytes;
-        float sc[KW / 8][4];
-        qk_any<D, KW, FP8>(q, kbase, key0, sc);
-        const int slot0 = i * kSparseTile + sub * kKeyTile + key0 + 2 * c;
-#pragma unroll
-        for (int nn = 0; nn < KW / 8; ++nn)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const bool ok = s_idx[slot0 + nn * 8 + (e & 1)] >= 0;
-                sc[nn][e] = ok ? sc[nn][e] * (e < 2 ? f_lo : f_hi) : -INFINITY;
-            }
-        st.template update<KW>(sc, vbase, key0);
-        __syncthreads();  // everyone is done with this stage before it is refilled
-        if (i + stages < ntl) {
-            gather_tile<D, FP8>(a.K, a.V, s_idx, i + stages, smem + stage * L::kStageBytes, kv_base);
-            cp_async_commit();
-        }
-    }
-    st.finish_rows();
     float* red = reinterpret_cast<float*>(smem);
-    stash_state<D, kSparseWarps, FP8>(st, warp, red, vscale);
+    if constexpr (TR) {
+        QTileT<D, FP8> q;
+        const int rq = row_q(g);
+        q.load(a.Q, rq >= 0 ? static_cast<int64_t>(rq) * D : -1);
+        const float f0 = a.scale_log2 * kscale * q.col_scale[0];
+        const float f1 = a.scale_log2 * kscale * q.col_scale[1];
+        OnlineSoftmaxT<D, FP8> st;
+        st.init();
+        for (int i = 0; i < ntl; ++i) {
+            cp_async_wait_upto(min(ntl, i + stages) - (i + 1));  // step i has landed
+            __syncthreads();
+            const int stage = i % stages;
+            const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes + sub * L::kSubBytes);
+            const uint32_t vbase = kbase + L::kTileBytes;
+            float sc[4];  // keys g, g + 8 of the warp's 16 for query heads 2c, 2c + 1
+            qk_t<D, FP8>(q, kbase, key0, sc);
+            const int slot = i * kSparseTile + sub * kKeyTile + key0 + g;
+            const bool v_lo = s_idx[slot] >= 0, v_hi = s_idx[slot + 8] >= 0;
+            sc[0] = v_lo ? sc[0] * f0 : -INFINITY;
+            sc[1] = v_lo ? sc[1] * f1 : -INFINITY;
+            sc[2] = v_hi ? sc[2] * f0 : -INFINITY;
+            sc[3] = v_hi ? sc[3] * f1 : -INFINITY;
+            st.update(sc, vbase, key0);
+            __syncthreads();  // everyone is done with this stage before it is refilled
+            if (i + stages < ntl) {
+                gather_tile<D, FP8>(a.K, a.V, s_idx, i + stages, smem + stage * L::kStageBytes, kv_base);
+                cp_async_commit();
+            }
+        }
+        st.finish_rows();
+        stash_state_t<D, kSparseWarps, FP8>(st, warp, red, vscale);
+    } else {
+        QTileOf<D, FP8> q;
+        {
+            const int r0 = row_q(g), r1 = row_q(g + 8);
+            q.load(a.Q, r0 >= 0 ? static_cast<int64_t>(r0) * D : -1, r1 >= 0 ? static_cast<int64_t>(r1) * D : -1);
+        }
+        const float f_lo = logit_factor<D, FP8>(q, 0, a.scale_log2, kscale);
+        const float f_hi = logit_factor<D, FP8>(q, 1, a.scale_log2, kscale);
+        OnlineSoftmax<D, FP8> st;
+        st.init();
+        for (int i = 0; i < ntl; ++i) {
+            cp_async_wait_upto(min(ntl, i + stages) - (i + 1));  // step i has landed
+            __syncthreads();
+            const int stage = i % stages;
+            const uint32_t kbase = smem_u32(smem + stage * L::kStageBytes + sub * L::kSubBytes);
+            const uint32_t vbase = kbase + L::kTileBytes;
+            float sc[KW / 8][4];
+            qk_any<D, KW, FP8>(q, kbase, key0, sc);
+            const int slot0 = i * kSparseTile + sub * kKeyTile + key0 + 2 * c;
+#pragma unroll
+            for (int nn = 0; nn < KW / 8; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool ok = s_idx[slot0 + nn * 8 + (e & 1)] >= 0;
+                    sc[nn][e] = ok ? sc[nn][e] * (e < 2 ? f_lo : f_hi) : -INFINITY;
+                }
+            st.template update<KW>(sc, vbase, key0);
+            __syncthreads();  // everyone is done with this stage before it is refilled
+            if (i + stages < ntl) {
+                gather_tile<D, FP8>(a.K, a.V, s_idx, i + stages, smem + stage * L::kStageBytes, kv_base);
+                cp_async_commit();
+            }
+        }
+        st.finish_rows();
+        stash_state<D, kSparseWarps, FP8>(st, warp, red, vscale);
+    }
     __syncthreads();
     merge_states<D, kSparseWarps>(red, tid, kSparseThreads, out, row_q);
     finish_row<D>(a, row, out_rows_q_base(a, b, h, t), smem);
 }
 
-template <int D, int MINB, bool FP8>
+template <int D, int MINB, bool FP8, bool TR>
 cudaError_t sparse_variant(const Plan& p, const SparseArgs& x, cudaStream_t st) {
-    auto kern = sparse_attn_kernel<D, MINB, FP8>;
+    auto kern = sparse_attn_kernel<D, MINB, FP8, TR>;
     const int bytes = SparseSmem<D, FP8>::bytes(x.stages, p.C4);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
@@ -180,7 +216,12 @@ cudaError_t sparse_variant(const Plan& p, const SparseArgs& x, cudaStream_t st) 
 
 template <int D, bool FP8>
 cudaError_t sparse_dispatch(const Plan& p, const SparseArgs& x, cudaStream_t st) {
-    return x.stages == 1 ? sparse_variant<D, 2, FP8>(p, x, st) : sparse_variant<D, 1, FP8>(p, x, st);
+    // at most 8 query heads per kv head: the transposed warp attention (HS2_TRANSPOSED=0: the
+    // 16-row form)
+    const char* env = std::getenv("HS2_TRANSPOSED");
+    if (p.G <= 8 && !(env && env[0] == '0'))
+        return x.stages == 1 ? sparse_variant<D, 2, FP8, true>(p, x, st) : sparse_variant<D, 1, FP8, true>(p, x, st);
+    return x.stages == 1 ? sparse_variant<D, 2, FP8, false>(p, x, st) : sparse_variant<D, 1, FP8, false>(p, x, st);
 }
 
 cudaError_t launch_sparse_attn(const Plan& p, const SparseArgs& a, cudaStream_t st) {

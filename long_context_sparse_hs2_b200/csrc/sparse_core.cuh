@@ -5,7 +5,7 @@
 // first 64-key sub-tile of a step, warps 4-7 the second).
 #pragma once
 
-#include "attn_core.cuh"
+#include "attn_core_t.cuh"
 
 namespace hs2 {
 
