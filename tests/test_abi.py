@@ -86,6 +86,22 @@ def test_prefill_selection_does_not_store_every_score_key(L, monkeypatch):
     assert 0 < bracketed < 2e9 and stored > 8.5e9, (bracketed, stored)
 
 
+def test_one_launch_decode_plan(L, monkeypatch):
+    # the one-launch decode step keeps one sparse partial per sweep split, so its plan needs more
+    # workspace than the kernel chain's; it is the default for short caches only
+    tiny = _dims(B=1, Hq=4, Hkv=1, d=64, N=2048, T=1, k=64, W=64)
+    long = _dims(B=1, Hq=64, Hkv=8, d=128, N=131072, T=1, k=4096, W=512)
+    sizes = {}
+    for env in (None, "0", "1"):
+        if env is None:
+            monkeypatch.delenv("HS2_FUSED_DECODE", raising=False)
+        else:
+            monkeypatch.setenv("HS2_FUSED_DECODE", env)
+        sizes[env] = (hs2.workspace_size(tiny), hs2.workspace_size(long))
+    assert sizes[None][0] == sizes["1"][0] > sizes["0"][0]      # tiny: one launch by default
+    assert sizes[None][1] == sizes["0"][1] < sizes["1"][1]      # 128K: the chain by default
+
+
 FAKE = 1 << 20  # a 256-byte-aligned non-null address; never dereferenced (checks fail first)
 
 
