@@ -140,9 +140,8 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_dims* dims, const void* Q_sparse, c
  * filtering candidates; HS2_TRANSPOSED=0 keeps the 16-row warp attention for decode row blocks;
  * HS2_DYN_SWEEP=1 / 0 forces the counter-scheduled sweep on / off (default: on for at least 128
  * key tiles per CTA); HS2_FUSED_DECODE=1 / 0 forces the one-launch decode step (T = 1) on / off
- * (default: caches of at most 8192 tokens); HS2_CLUSTER_TAIL=1 runs the decode tail after the
- * sweep (T*G <= 16) as one thread-block cluster per selection row instead of the three-kernel
- * chain.  The plan, and so the workspace size, also follows the current device's SM count. */
+ * (default: caches of at most 8192 tokens).  The plan, and so the workspace size, also follows
+ * the current device's SM count. */
 HS2_API hs2_status hs2_step(const hs2_dims* dims, const void* Q_full, const void* Q_sparse,
                     const void* K, const void* V, const int32_t* pos,
                     void* O_full, void* O_sparse, float* LSE_full, float* LSE_sparse,

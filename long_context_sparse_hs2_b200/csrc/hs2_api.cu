@@ -434,42 +434,6 @@ hs2_status run_sparse(const Plan& p, const void* Qs, const KvView& kv, const int
     return HS2_OK;
 }
 
-// Selection and sparse layer from the kept logits in one cluster kernel; *done = false when the
-// shape does not fit it (nothing launched).
-hs2_status run_tail(const Plan& p, const void* Qs, const KvView& kv, const int32_t* pos, void* O_full,
-                    void* O_sparse, float* LSE_full, float* LSE_sparse, int32_t* idx, int32_t* cnt, const Ws& w,
-                    cudaStream_t st, bool* done) {
-    *done = false;
-    // HS2_CLUSTER_TAIL=1: the cluster kernel wherever it fits; otherwise the kernel chain, which
-    // measured faster at every decode shape (see launch_tail)
-    const char* env = std::getenv("HS2_CLUSTER_TAIL");
-    if (!env || env[0] != '1') return HS2_OK;
-    const bool force = env && env[0] == '1';
-    TailArgs t{};
-    t.logits = w.at<float>(p.off_logits);
-    t.pf_ml = w.at<float2>(p.off_pf_ml);
-    t.pf_acc = w.at<float>(p.off_pf_acc);
-    t.S1 = p.S1;
-    t.Qs = static_cast<const uint16_t*>(Qs);
-    t.K = kv.K;
-    t.V = kv.V;
-    t.kv = kv.src;
-    t.pos = pos;
-    t.B = p.B; t.Hq = p.Hq; t.Hkv = p.Hkv; t.T = p.T; t.N = p.N; t.k = p.k; t.W = p.W;
-    t.scale_log2 = scale_log2(p);
-    t.O_full = static_cast<uint16_t*>(O_full);
-    t.LSE_full = LSE_full;
-    t.O_sparse = static_cast<uint16_t*>(O_sparse);
-    t.LSE_sparse = LSE_sparse;
-    t.idx = idx;
-    t.cnt = cnt;
-    t.cand = w.at<unsigned long long>(p.off_cand);
-    t.cand_cap = p.cand_cap;
-    t.status = w.at<unsigned>(p.off_status);
-    HS2_TRY(launch_tail(p, t, st, force, done));
-    return HS2_OK;
-}
-
 // The one-launch decode step; *done = false when its grid does not fit on the device at once
 // (nothing launched).  The counters and histograms must have been cleared before.
 hs2_status run_fused(const Plan& p, const void* Qf, const void* Qs, const KvView& kv, const int32_t* pos,
@@ -514,11 +478,6 @@ hs2_status run_step(const Plan& p, const void* Qf, const void* Qs, const KvView&
     hs2_status s = run_full(p, Qf, kv, pos, O_full, LSE_full, w, p.mat_logits, !p.mat_logits, p.off_meta,
                             p.zero_bytes, st, first_pdl);
     if (s != HS2_OK) return s;
-    if (p.mat_logits && p.cand_cap >= p.N) {
-        bool done = false;
-        s = run_tail(p, Qs, kv, pos, O_full, O_sparse, LSE_full, LSE_sparse, idx, cnt, w, st, &done);
-        if (s != HS2_OK || done) return s;
-    }
     s = p.mat_logits ? run_select_kept(p, pos, O_full, LSE_full, idx, cnt, w, st)
                      : run_select_sweep(p, Qf, kv, LSE_full, pos, idx, cnt, w, st);
     if (s != HS2_OK) return s;

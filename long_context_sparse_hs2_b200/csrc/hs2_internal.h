@@ -199,30 +199,6 @@ struct FusedArgs {          // the selection and sparse layer of the one-launch 
     float* ps_acc;         // [S][rows_q][D]
 };
 
-struct TailArgs {           // the decode step after the sweep, one cluster per selection row (k_tail.cu)
-    const float* logits;   // [rows_kv][N][G] base-2 logits of the sweep
-    const float2* pf_ml;   // full-attention split partials [S1][rows_q]
-    const float* pf_acc;   // [S1][rows_q][D]
-    int S1;
-    const uint16_t* Qs;    // Q_sparse [B][Hq][T][D]
-    const void* K;         // the cache (contiguous or pool), bf16 or E4M3 codes
-    const void* V;
-    KvSrc kv;
-    const int32_t* pos;    // [B][T]
-    int B, Hq, Hkv, T, N, k, W;
-    int stages;            // gather ring depth (set by the launcher)
-    float scale_log2;
-    uint16_t* O_full;
-    float* LSE_full;
-    uint16_t* O_sparse;
-    float* LSE_sparse;
-    int32_t* idx;          // [rows_kv][k+W]
-    int32_t* cnt;          // [rows_kv]
-    unsigned long long* cand;  // [rows_kv][cand_cap] candidate composites of the threshold bucket
-    int64_t cand_cap;
-    unsigned* status;
-};
-
 struct TopkArgs {
     const uint32_t* keys;  // [rows][kstride] (the sample keys for the bracket kernel)
     int64_t kstride;
@@ -317,10 +293,6 @@ cudaError_t launch_topk_bracket(const Plan& p, const TopkArgs& a, cudaStream_t s
 // ... and, after the filtering sweep, the exact selection from the candidate list (an exact
 // rescoring of the row where the bracket did not hold).
 cudaError_t launch_topk_finalize(const Plan& p, const TopkArgs& a, cudaStream_t st);
-// The decode tail as one cluster kernel; *launched = false (nothing launched, cudaSuccess) when
-// the shape does not fit its plan, or (unless force) when the kernel chain measured faster for
-// it -- the caller then runs score_hist, topk_select, sparse_attn.
-cudaError_t launch_tail(const Plan& p, const TailArgs& a, cudaStream_t st, bool force, bool* launched);
 cudaError_t launch_topk_select(const Plan& p, const TopkArgs& a, cudaStream_t st);
 // The one-launch decode step (T = 1): sweep, selection and sparse layer in one cooperative grid
 // of p.S1 x rows_kv CTAs.  *launched = false (nothing launched, cudaSuccess) when the grid does

@@ -1,5 +1,5 @@
-// The gathered-attention core of the sparse layer (sm_100a), shared by the sparse-attention
-// kernel and the decode tail: selected K/V rows are gathered with 16-byte cp.async into the
+// The gathered-attention core of the sparse layer (sm_100a), used by the sparse-attention
+// kernel: selected K/V rows are gathered with 16-byte cp.async into the
 // same swizzled tile layout the TMA path writes (bf16 or FP8 E4M3 tiles), a ring of up to three
 // 128-key steps in flight, and 8 warps run the warp attention core on them (warps 0-3 take the
 // first 64-key sub-tile of a step, warps 4-7 the second).

@@ -251,15 +251,13 @@ def test_repeated_calls_reuse_workspace():
 TAIL_CASES = [c for c in CASES if c[5] * (c[1] // c[2]) <= 16]
 
 
-@pytest.mark.parametrize("path", ["fused", "cluster", "chain"])
+@pytest.mark.parametrize("path", ["fused", "chain"])
 @pytest.mark.parametrize("case", TAIL_CASES, ids=[str(c) for c in TAIL_CASES])
 def test_decode_tail_paths_match_oracle(case, path, monkeypatch):
-    # the decode tail after the sweep: the cluster tail (selection + sparse layer in one cluster
-    # kernel), the kernel chain (score_hist -> topk_select -> sparse_attn), and, for T = 1, the
-    # whole step in one cooperative launch (HS2_FUSED_DECODE=1; the default for short caches)
+    # the decode tail after the sweep: the kernel chain (score_hist -> topk_select ->
+    # sparse_attn), and, for T = 1, the whole step in one cooperative launch
+    # (HS2_FUSED_DECODE=1; the default for short caches)
     monkeypatch.setenv("HS2_FUSED_DECODE", "1" if path == "fused" else "0")
-    if path != "fused":
-        monkeypatch.setenv("HS2_CLUSTER_TAIL", "1" if path == "cluster" else "0")
     B, Hq, Hkv, d, N, T, k, W = case
     inp = make_inputs(B, Hq, Hkv, d, N, T, k, W, seed=hash(case) % 1000 + 7, needles=4)
     hs2.trace_enable(True)
@@ -268,10 +266,8 @@ def test_decode_tail_paths_match_oracle(case, path, monkeypatch):
     hs2.trace_enable(False)
     if path == "fused":
         assert ("decode_fused" in kernels) == (T == 1), kernels
-    elif path == "cluster":
-        assert "select_sparse_cluster" in kernels and "topk_select" not in kernels, kernels
     else:
-        assert "select_sparse_cluster" not in kernels and "topk_select" in kernels, kernels
+        assert "decode_fused" not in kernels and "topk_select" in kernels, kernels
     compare_step(inp, res)
 
 
